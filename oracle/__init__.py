@@ -1,0 +1,154 @@
+"""fp64 CPU oracle for token-level dynamic local-global attention (LoGo / L2A).
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
+benchmark's CPU-baseline leg may import this package.  The library's product
+path never does: it has no CPU fallback.
+
+The arithmetic lives in ``logo_oracle.c`` (plain loops in double precision);
+this module only marshals torch CPU tensors into it.  Each function cites the
+passage of the pages it follows in the C source.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SO = os.path.join(_HERE, "liblogo_oracle.so")
+_SRC = os.path.join(_HERE, "logo_oracle.c")
+_lock = threading.Lock()
+_lib = None
+
+_p = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+_dbl = ctypes.c_double
+
+
+def build() -> str:
+    """Compile the oracle with the Makefile beside it (gcc, OpenMP if available)."""
+    subprocess.run(["make", "-s", "-C", _HERE], check=True)
+    return _SO
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if (not os.path.exists(_SO)) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+            build()
+        lib = ctypes.CDLL(_SO)
+        lib.oracle_num_selected.argtypes = [_dbl, _i64]
+        lib.oracle_num_selected.restype = _i64
+        lib.oracle_select.argtypes = [_p, _i64, _dbl, _p]
+        lib.oracle_select.restype = _i64
+        lib.oracle_forward.argtypes = [_p, _p, _p, _p, _p, _int, _int, _int, _i64, _int, _i64,
+                                       _dbl, _dbl, _p, _p, _p, _p, _p]
+        lib.oracle_forward.restype = _i64
+        lib.oracle_rows.argtypes = [_p, _p, _p, _p, _p, _int, _int, _int, _i64, _int, _i64, _dbl,
+                                    _i64, _p, _p, _p, _p, _p, _p, _p]
+        lib.oracle_rows.restype = None
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = _int
+        _lib = lib
+        return lib
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _bits(x: torch.Tensor) -> torch.Tensor:
+    assert x.dtype == torch.bfloat16 and x.device.type == "cpu"
+    return x.contiguous().view(torch.int16)
+
+
+def num_selected(ratio: float, length: int) -> int:
+    """k = ceil(ratio * length) with fp noise snapped (see logo_oracle.c)."""
+    return int(_load().oracle_num_selected(float(ratio), int(length)))
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def select(g: torch.Tensor, ratio: float) -> torch.Tensor:
+    """Selected positions (ascending) of one sequence's fp32 gate logits."""
+    g = g.detach().to(torch.float32).contiguous()
+    k = num_selected(ratio, g.numel())
+    out = torch.empty(max(k, 1), dtype=torch.int32)
+    got = _load().oracle_select(_ptr(g), g.numel(), float(ratio), _ptr(out))
+    assert got == k
+    return out[:k].clone()
+
+
+def _geometry(q, k, cu_seqlens):
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    if cu_seqlens is not None:
+        assert B == 1
+        nseq = cu_seqlens.numel() - 1
+    else:
+        nseq = B
+    return B, Hq, Hkv, L, d, nseq
+
+
+def forward(q, k, v, g, window: int, ratio: float, scale: float = 0.0, cu_seqlens=None,
+            want_branches: bool = False):
+    """Whole forward pass in fp64.
+
+    q: bf16 [B, Hq, L, d]; k, v: bf16 [B, Hkv, L, d]; g: fp32 [B, L].
+    Varlen: B == 1, L == T and ``cu_seqlens`` int32 [nseq + 1].
+    Returns a dict with ``out`` (fp64 [B, Hq, L, d]), ``sel_idx`` (int32, the
+    sequences' ascending lists back to back), ``cu_sel`` (int32 [nseq + 1])
+    and, if ``want_branches``, ``local`` and ``global`` (global is 0 on rows
+    that are not selected).
+    """
+    B, Hq, Hkv, L, d, nseq = _geometry(q, k, cu_seqlens)
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    g32 = g.detach().to(torch.float32).contiguous()
+    cu = None if cu_seqlens is None else cu_seqlens.to(torch.int32).contiguous()
+    lens = [L] * B if cu is None else (cu[1:] - cu[:-1]).tolist()
+    cap = max(1, sum(num_selected(ratio, n) for n in lens))
+    out = torch.empty(B, Hq, L, d, dtype=torch.float64)
+    loc = torch.empty_like(out) if want_branches else None
+    glo = torch.empty_like(out) if want_branches else None
+    sel = torch.empty(cap, dtype=torch.int32)
+    cu_sel = torch.empty(nseq + 1, dtype=torch.int32)
+    total = _load().oracle_forward(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(g32), _ptr(cu), nseq, Hq, Hkv,
+                                   L, d, int(window), float(ratio), float(scale), _ptr(out),
+                                   _ptr(loc), _ptr(glo), _ptr(sel), _ptr(cu_sel))
+    res = {"out": out, "sel_idx": sel[:total].clone(), "cu_sel": cu_sel}
+    if want_branches:
+        res["local"] = loc
+        res["global"] = glo
+    return res
+
+
+def rows(q, k, v, g, window: int, seq, head, pos, selected, scale: float = 0.0, cu_seqlens=None):
+    """fp64 outputs of a sample of rows: (local, global, merged), each [n, d].
+
+    ``seq``, ``head``, ``pos`` (relative to the sequence start) and
+    ``selected`` (0/1, from :func:`select`) are 1-D sequences of length n.
+    """
+    B, Hq, Hkv, L, d, nseq = _geometry(q, k, cu_seqlens)
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    g32 = g.detach().to(torch.float32).contiguous()
+    cu = None if cu_seqlens is None else cu_seqlens.to(torch.int32).contiguous()
+    seq_t = torch.as_tensor(seq, dtype=torch.int32).contiguous()
+    head_t = torch.as_tensor(head, dtype=torch.int32).contiguous()
+    pos_t = torch.as_tensor(pos, dtype=torch.int64).contiguous()
+    sel_t = torch.as_tensor(selected, dtype=torch.uint8).contiguous()
+    n = seq_t.numel()
+    loc = torch.empty(n, d, dtype=torch.float64)
+    glo = torch.empty(n, d, dtype=torch.float64)
+    out = torch.empty(n, d, dtype=torch.float64)
+    _load().oracle_rows(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(g32), _ptr(cu), nseq, Hq, Hkv, L, d,
+                        int(window), float(scale), n, _ptr(seq_t), _ptr(head_t), _ptr(pos_t),
+                        _ptr(sel_t), _ptr(loc), _ptr(glo), _ptr(out))
+    return loc, glo, out

@@ -1,0 +1,355 @@
+/*
+ * logo_oracle.c -- plain, slow fp64 CPU oracle for the forward pass of
+ * token-level dynamic local-global attention (LoGo / L2A).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the library's product path may link,
+ * load or call this file: it exists so that the tests, the smoke check and the
+ * benchmark's CPU-baseline leg can compare the CUDA kernels against a
+ * definition a reader can check by eye.  It shares no code, header, table or
+ * helper with the CUDA library.
+ *
+ * What it computes (sources are the pages' titles and sections):
+ *   - "LoGo: Token-Level Dynamic Local-Global Attention", Abstract: every
+ *     token gets local attention over a restricted window; a learned gate
+ *     turns on full-context (global) attention for a subset of tokens; a
+ *     budget controller keeps a target global ratio.
+ *   - "Learning When to Attend", section "The Architecture of Conditional
+ *     Attention": local attention over a fixed recent window for all tokens,
+ *     then exact attention over the full context for a sparse subset of query
+ *     tokens only.
+ *   - "Local-global attention", Variants, "Alternating sliding-window and
+ *     global layers (Gemma 2)": both kinds are causal; the local kind drops
+ *     keys more than the window back.
+ *   - "Local-global attention", Implementation sketch, notes, "Packed examples
+ *     (LongT5)": packed examples must not attend to one another.
+ *
+ * Readings taken where the pages are silent (each is listed in the design
+ * notes of the repository):
+ *   window      key j is in the local window of query i iff 0 <= i - j < W
+ *               (W keys including the query itself);
+ *   budget      k = ceil(ratio * len) per sequence (with fp noise snapped, see
+ *               oracle_num_selected), chosen as the k largest gate logits,
+ *               ties to the lower index, -0 equal to +0, NaN below -inf;
+ *               one selection per sequence, shared by every head;
+ *   global      exact causal attention over positions 0..i of the sequence;
+ *   merge       o_i = local_i + sigmoid(g_i) * global_i for selected i,
+ *               o_i = local_i otherwise;
+ *   scale       softmax scale 1/sqrt(d) unless the caller passes scale > 0;
+ *   GQA         query head h reads key/value head h / (Hq / Hkv).
+ *
+ * Precision: inputs are bf16 (passed as raw uint16 bit patterns) and gate
+ * logits fp32; both are widened exactly to double, and every sum, max,
+ * exponential and division is done in double.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ---- scalar helpers --------------------------------------------------- */
+
+/* bf16 -> double, exact: a bf16 value is the top half of an fp32 value. */
+static double bf16_bits_to_double(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+/*
+ * Budget: the number of query tokens that take the global branch in a
+ * sequence of `len` tokens at target ratio `ratio` ("LoGo", Abstract: a
+ * budget controller keeps a target global ratio; "Learning When to Attend",
+ * "The Architecture of Conditional Attention": about 20% of tokens).
+ * Reading: k = ceil(ratio * len).  The product is formed in double; when it
+ * lies within 1e-9 (relative, at least absolute 1e-9) of an integer it is
+ * taken as that integer, so that 0.2 * 5 = 1.0000000000000002 gives 1, not 2.
+ * The result is clamped to [0, len].
+ */
+int64_t oracle_num_selected(double ratio, int64_t len)
+{
+    if (len <= 0 || !(ratio > 0.0)) return 0;
+    double x = ratio * (double)len;
+    double r = nearbyint(x);
+    double tol = 1e-9 * (x > 1.0 ? x : 1.0);
+    double kk = (fabs(x - r) <= tol) ? r : ceil(x);
+    if (kk < 0.0) kk = 0.0;
+    if (kk > (double)len) kk = (double)len;
+    return (int64_t)kk;
+}
+
+/* ---- selection -------------------------------------------------------- */
+
+typedef struct {
+    float g;
+    int32_t idx;
+} gate_item;
+
+/*
+ * Order used by the budget rule: larger logit first; equal logits (and -0 vs
+ * +0, which compare equal as floats) by lower index; NaN after every number,
+ * NaNs among themselves by lower index.
+ */
+static int gate_order(const void *pa, const void *pb)
+{
+    const gate_item *a = (const gate_item *)pa;
+    const gate_item *b = (const gate_item *)pb;
+    int a_nan = isnan(a->g), b_nan = isnan(b->g);
+    if (a_nan != b_nan) return a_nan ? 1 : -1;
+    if (!a_nan) {
+        if (a->g > b->g) return -1;
+        if (a->g < b->g) return 1;
+    }
+    return (a->idx < b->idx) ? -1 : (a->idx > b->idx ? 1 : 0);
+}
+
+static int ascending_i32(const void *pa, const void *pb)
+{
+    int32_t a = *(const int32_t *)pa, b = *(const int32_t *)pb;
+    return (a > b) - (a < b);
+}
+
+/*
+ * Select the k = oracle_num_selected(ratio, len) tokens of one sequence:
+ * sort all positions by the order above, keep the first k, and return them
+ * in ascending position order.  `out` holds at least k entries.  Returns k.
+ */
+int64_t oracle_select(const float *g, int64_t len, double ratio, int32_t *out)
+{
+    int64_t k = oracle_num_selected(ratio, len);
+    if (k == 0) return 0;
+    gate_item *items = (gate_item *)malloc(sizeof(gate_item) * (size_t)len);
+    for (int64_t i = 0; i < len; ++i) {
+        items[i].g = g[i];
+        items[i].idx = (int32_t)i;
+    }
+    qsort(items, (size_t)len, sizeof(gate_item), gate_order);
+    for (int64_t i = 0; i < k; ++i) out[i] = items[i].idx;
+    free(items);
+    qsort(out, (size_t)k, sizeof(int32_t), ascending_i32);
+    return k;
+}
+
+/* ---- attention for one query row -------------------------------------- */
+
+/*
+ * Exact softmax attention of one query row over the keys j_lo..j_hi
+ * (inclusive) of one key/value head:
+ *   s_j = scale * <q, k_j>,  w_j = exp(s_j - max_j s_j),
+ *   out = sum_j w_j v_j / sum_j w_j.
+ * `q`, `kh`, `vh` point at the query row and at row 0 of the key and value
+ * sequences; rows are d elements apart.  `s` is scratch for j_hi - j_lo + 1
+ * doubles.
+ */
+static void attend_row(const uint16_t *q, const uint16_t *kh, const uint16_t *vh,
+                       int64_t j_lo, int64_t j_hi, int d, double scale,
+                       double *s, double *out)
+{
+    int64_t n = j_hi - j_lo + 1;
+    double m = -INFINITY;
+    for (int64_t t = 0; t < n; ++t) {
+        const uint16_t *kr = kh + (j_lo + t) * (int64_t)d;
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c) dot += bf16_bits_to_double(q[c]) * bf16_bits_to_double(kr[c]);
+        s[t] = scale * dot;
+        if (s[t] > m) m = s[t];
+    }
+    double den = 0.0;
+    for (int c = 0; c < d; ++c) out[c] = 0.0;
+    for (int64_t t = 0; t < n; ++t) {
+        double w = exp(s[t] - m);
+        den += w;
+        const uint16_t *vr = vh + (j_lo + t) * (int64_t)d;
+        for (int c = 0; c < d; ++c) out[c] += w * bf16_bits_to_double(vr[c]);
+    }
+    for (int c = 0; c < d; ++c) out[c] /= den;
+}
+
+/* ---- problem geometry ------------------------------------------------- */
+
+/*
+ * Tensors are [B, H, L, d] (fixed length, cu_seqlens == NULL, nseq == B), or
+ * packed [1, H, T, d] with sequence s at rows cu_seqlens[s] .. cu_seqlens[s+1]
+ * of every head (varlen, B == 1, L == T).
+ */
+typedef struct {
+    const uint16_t *q, *k, *v;
+    const float *g;
+    const int32_t *cu_seqlens;
+    int nseq, Hq, Hkv, d;
+    int64_t L; /* rows per head slab: L (fixed) or T (varlen) */
+    int64_t W;
+    double scale;
+} problem;
+
+static int64_t seq_start(const problem *p, int s)
+{
+    return p->cu_seqlens ? (int64_t)p->cu_seqlens[s] : 0;
+}
+
+static int64_t seq_len(const problem *p, int s)
+{
+    return p->cu_seqlens ? (int64_t)(p->cu_seqlens[s + 1] - p->cu_seqlens[s]) : p->L;
+}
+
+/* Pointer to row `row` (absolute within the slab) of head `h` of batch `b`. */
+static const uint16_t *row_ptr(const uint16_t *base, int64_t b, int64_t H, int64_t h,
+                               int64_t L, int64_t row, int d)
+{
+    return base + (((b * H + h) * L) + row) * (int64_t)d;
+}
+
+/*
+ * One output row: sequence s, query head h, position i (relative to the
+ * sequence start).  Writes the local row, and, if `want_global`, the global
+ * row.  Either output pointer may be NULL.
+ */
+static void compute_row(const problem *p, int s, int h, int64_t i, int want_global,
+                        double *scratch, double *loc, double *glo)
+{
+    int G = p->Hq / p->Hkv;
+    int hk = h / G;
+    int64_t b = p->cu_seqlens ? 0 : s;
+    int64_t s0 = seq_start(p, s);
+    const uint16_t *qr = row_ptr(p->q, b, p->Hq, h, p->L, s0 + i, p->d);
+    const uint16_t *kh = row_ptr(p->k, b, p->Hkv, hk, p->L, s0, p->d);
+    const uint16_t *vh = row_ptr(p->v, b, p->Hkv, hk, p->L, s0, p->d);
+    if (loc) {
+        int64_t j_lo = i - p->W + 1;
+        if (j_lo < 0) j_lo = 0;
+        attend_row(qr, kh, vh, j_lo, i, p->d, p->scale, scratch, loc);
+    }
+    if (want_global && glo) attend_row(qr, kh, vh, 0, i, p->d, p->scale, scratch, glo);
+}
+
+static double default_scale(double scale, int d) { return scale > 0.0 ? scale : 1.0 / sqrt((double)d); }
+
+/* ---- public entry points ---------------------------------------------- */
+
+/*
+ * Full forward pass.
+ *   out        [B, Hq, L, d] doubles: the merged output o.
+ *   out_local  (may be NULL) [B, Hq, L, d]: the local branch for every row.
+ *   out_global (may be NULL) [B, Hq, L, d]: the global branch on selected
+ *              rows, 0 elsewhere.
+ *   sel_idx    the selected positions, sequence after sequence, each
+ *              sequence ascending; capacity sum_s k_s.
+ *   cu_sel     [nseq + 1] offsets of each sequence's list in sel_idx.
+ * Returns the total number of selected tokens.
+ */
+int64_t oracle_forward(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                       const int32_t *cu_seqlens, int nseq, int Hq, int Hkv, int64_t L, int d,
+                       int64_t W, double ratio, double scale, double *out, double *out_local,
+                       double *out_global, int32_t *sel_idx, int32_t *cu_sel)
+{
+    problem p = {q, k, v, g, cu_seqlens, nseq, Hq, Hkv, d, L, W, default_scale(scale, d)};
+    int64_t B = cu_seqlens ? 1 : nseq;
+    int64_t total_rows = B * (int64_t)Hq * L;
+
+    /* Selection, one sequence at a time; the flag marks selected rows. */
+    unsigned char *flag = (unsigned char *)calloc((size_t)(B * L), 1);
+    int64_t off = 0;
+    cu_sel[0] = 0;
+    for (int s = 0; s < nseq; ++s) {
+        int64_t b = cu_seqlens ? 0 : s;
+        int64_t s0 = seq_start(&p, s), len = seq_len(&p, s);
+        int64_t ks = oracle_select(g + b * L + s0, len, ratio, sel_idx + off);
+        for (int64_t t = 0; t < ks; ++t) flag[b * L + s0 + sel_idx[off + t]] = 1;
+        off += ks;
+        cu_sel[s + 1] = (int32_t)off;
+    }
+
+    memset(out, 0, sizeof(double) * (size_t)(total_rows * d));
+    if (out_local) memset(out_local, 0, sizeof(double) * (size_t)(total_rows * d));
+    if (out_global) memset(out_global, 0, sizeof(double) * (size_t)(total_rows * d));
+
+    /* Every (sequence, head, position) row is independent. */
+    for (int s = 0; s < nseq; ++s) {
+        int64_t b = cu_seqlens ? 0 : s;
+        int64_t s0 = seq_start(&p, s), len = seq_len(&p, s);
+#pragma omp parallel
+        {
+            double *scratch = (double *)malloc(sizeof(double) * (size_t)(len > 0 ? len : 1));
+            double *loc = (double *)malloc(sizeof(double) * (size_t)d);
+            double *glo = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 16) collapse(2)
+            for (int h = 0; h < Hq; ++h) {
+                for (int64_t i = 0; i < len; ++i) {
+                    int sel = flag[b * L + s0 + i];
+                    compute_row(&p, s, h, i, sel, scratch, loc, glo);
+                    double gs = sel ? sigmoid((double)g[b * L + s0 + i]) : 0.0;
+                    int64_t r = ((b * Hq + h) * L + s0 + i) * (int64_t)d;
+                    for (int c = 0; c < d; ++c) {
+                        out[r + c] = loc[c] + (sel ? gs * glo[c] : 0.0);
+                        if (out_local) out_local[r + c] = loc[c];
+                        if (out_global && sel) out_global[r + c] = glo[c];
+                    }
+                }
+            }
+            free(scratch);
+            free(loc);
+            free(glo);
+        }
+    }
+    free(flag);
+    return off;
+}
+
+/*
+ * A sample of rows, for problems too large to run whole.  Row t is
+ * (seq[t], head[t], pos[t]) with pos relative to the sequence start;
+ * selected[t] says whether that position is in the sequence's selection
+ * (taken from oracle_select by the caller).  Writes d doubles per row into
+ * each non-NULL output: the local branch, the global branch (0 when not
+ * selected) and the merged output.
+ */
+void oracle_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                 const int32_t *cu_seqlens, int nseq, int Hq, int Hkv, int64_t L, int d, int64_t W,
+                 double scale, int64_t n, const int32_t *seq, const int32_t *head,
+                 const int64_t *pos, const unsigned char *selected, double *out_local,
+                 double *out_global, double *out)
+{
+    problem p = {q, k, v, g, cu_seqlens, nseq, Hq, Hkv, d, L, W, default_scale(scale, d)};
+    int64_t maxlen = 1;
+    for (int s = 0; s < nseq; ++s)
+        if (seq_len(&p, s) > maxlen) maxlen = seq_len(&p, s);
+#pragma omp parallel
+    {
+        double *scratch = (double *)malloc(sizeof(double) * (size_t)maxlen);
+        double *loc = (double *)malloc(sizeof(double) * (size_t)d);
+        double *glo = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < n; ++t) {
+            int s = seq[t];
+            int64_t b = cu_seqlens ? 0 : s;
+            int sel = selected[t] != 0;
+            compute_row(&p, s, head[t], pos[t], sel, scratch, loc, glo);
+            double gs = sel ? sigmoid((double)g[b * L + seq_start(&p, s) + pos[t]]) : 0.0;
+            for (int c = 0; c < d; ++c) {
+                if (out_local) out_local[t * d + c] = loc[c];
+                if (out_global) out_global[t * d + c] = sel ? glo[c] : 0.0;
+                if (out) out[t * d + c] = loc[c] + (sel ? gs * glo[c] : 0.0);
+            }
+        }
+        free(scratch);
+        free(loc);
+        free(glo);
+    }
+}
+
+/* Number of threads the oracle runs on (for reporting). */
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,99 @@
+"""The oracle's pins must catch plausible mistakes (CPU only).
+
+Each case copies the oracle's C source to a temporary directory, plants one
+mistake in the copy (a window off by one, a wrong sign, a wrong head index, a
+transposed operand, a reversed tie-break, ...), builds it, and checks that at
+least one pin of tests/test_oracle_pins.py fails against it.  The oracle in
+the repository is never modified.
+"""
+import contextlib
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "logo_oracle.c")
+
+MUTANTS = {
+    "window_off_by_one": ("int64_t j_lo = i - p->W + 1;", "int64_t j_lo = i - p->W;"),
+    "merge_sign": ("out[r + c] = loc[c] + (sel ? gs * glo[c] : 0.0);",
+                   "out[r + c] = loc[c] - (sel ? gs * glo[c] : 0.0);"),
+    "gqa_head_map": ("int hk = h / G;", "int hk = h % p->Hkv;"),
+    "scores_read_v": ("const uint16_t *kr = kh + (j_lo + t) * (int64_t)d;",
+                      "const uint16_t *kr = vh + (j_lo + t) * (int64_t)d;"),
+    "tie_break_upper": ("return (a->idx < b->idx) ? -1 : (a->idx > b->idx ? 1 : 0);",
+                        "return (a->idx > b->idx) ? -1 : (a->idx < b->idx ? 1 : 0);"),
+    "nan_on_top": ("if (a_nan != b_nan) return a_nan ? 1 : -1;",
+                   "if (a_nan != b_nan) return a_nan ? -1 : 1;"),
+    "sigmoid_sign": ("return 1.0 / (1.0 + exp(-x));", "return 1.0 / (1.0 + exp(x));"),
+    "budget_floor": ("double kk = (fabs(x - r) <= tol) ? r : ceil(x);",
+                     "double kk = (fabs(x - r) <= tol) ? r : floor(x);"),
+    "budget_no_snap": ("double kk = (fabs(x - r) <= tol) ? r : ceil(x);", "double kk = ceil(x);"),
+    "scale_one_over_d": ("return scale > 0.0 ? scale : 1.0 / sqrt((double)d);",
+                         "return scale > 0.0 ? scale : 1.0 / (double)d;"),
+    "denominator_dropped_term": ("den += w;", "den += (t == 0) ? 0.0 : w;"),
+    "global_not_full_prefix": ("attend_row(qr, kh, vh, 0, i, p->d, p->scale, scratch, glo);",
+                               "attend_row(qr, kh, vh, i > 0 ? 1 : 0, i, p->d, p->scale, scratch, glo);"),
+}
+
+PINS = [
+    pins.test_num_selected_golden,
+    pins.test_select_golden,
+    lambda: [pins.test_select_bruteforce_ties_nan_inf(s) for s in range(4)],
+    lambda: [pins.test_oracle_vs_dense_masks(s) for s in pins.SHAPES],
+    pins.test_oracle_vs_dense_masks_varlen,
+    pins.test_oracle_vs_sdpa,
+    pins.test_closed_form_uniform_weights,
+    pins.test_closed_form_weights_one_e_e2,
+    pins.test_ratio_one_full_window_is_gated_causal,
+]
+
+
+@contextlib.contextmanager
+def swapped_oracle(so_path):
+    saved = oracle._lib
+    oracle._lib = None
+    real_so = oracle._SO
+    real_src = oracle._SRC
+    try:
+        oracle._SO = so_path
+        oracle._SRC = so_path  # mtime check passes: no rebuild
+        oracle._load()
+        yield
+    finally:
+        oracle._lib = saved
+        oracle._SO = real_so
+        oracle._SRC = real_src
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not found exactly once: {old}"
+    mutated = tmp_path / "mutant.c"
+    mutated.write_text(src.replace(old, new))
+    so = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O1", "-fPIC", "-std=gnu11", "-shared", "-o", str(so), str(mutated), "-lm"],
+                   check=True)
+    caught = []
+    with swapped_oracle(str(so)):
+        for pin in PINS:
+            try:
+                pin()
+            except AssertionError:
+                caught.append(getattr(pin, "__name__", "pin"))
+    assert caught, f"no pin caught the planted mistake {name}"
+
+
+def test_unmutated_copy_passes_every_pin(tmp_path):
+    so = tmp_path / "libcopy.so"
+    subprocess.run(["gcc", "-O1", "-fPIC", "-std=gnu11", "-shared", "-o", str(so), SRC, "-lm"],
+                   check=True)
+    with swapped_oracle(str(so)):
+        for pin in PINS:
+            pin()
