@@ -1,0 +1,373 @@
+"""Benchmark: forward pass of token-level dynamic local-global attention on B200.
+
+Workload (N = 1): B=1, Hq=32, Hkv=8 (GQA), L=32768, d=128, W=4096, ratio 0.2,
+bf16 N(0,1) Q/K/V, fp32 N(0,1) gate logits (seeded, synthetic).  One step is
+one pass of the whole hot path: selection, local attention, query-sparse
+global attention with the fused gated merge, launched through the C ABI on one
+stream.  With --gpus N (torchrun), every rank runs its own independent
+sequence (seed = rank): weak scaling, no collective on the data path; the
+timed region is bracketed by barriers and the reported time is the max over
+ranks.
+
+Printed: one JSON line (rank 0).  ``--impl reference`` instead times the fp64
+CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import random
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+import torch.distributed as dist  # noqa: E402
+
+METRIC = "LoGo fwd tokens/s & useful TFLOP/s (frac of bf16 peak) at L=32K, 20% global"
+WORKLOAD = "c32k"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def traffic_record():
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            return json.load(f)
+    except Exception:
+        return {}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+        except Exception:
+            uuid = None
+        self.uuid = uuid
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 8:
+                self.samples.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        if not self.samples:
+            return None
+        sm = []
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        max_mhz = None
+        for s in self.samples:
+            try:
+                sm.append(float(s[0]))
+                max_mhz = float(s[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, s[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        busy = [x for x in sm if max_mhz is None or x > 0.3 * max_mhz] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max_mhz, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_baseline(w, seconds_target=15.0, seed=0):
+    """The fp64 oracle on a bounded sample of the workload: whole tokens (all heads,
+    local branch, global branch where selected, merge), tokens/s on the host cores."""
+    import oracle
+
+    sel = set(oracle.select(w.g[0], w.ratio).tolist())
+    rng = random.Random(seed)
+    n_tok = 2
+    elapsed = 0.0
+    done = 0
+    while elapsed < seconds_target:
+        toks = [rng.randrange(w.L) for _ in range(n_tok)]
+        seq, head, pos, flag = [], [], [], []
+        for t in toks:
+            for h in range(w.Hq):
+                seq.append(0)
+                head.append(h)
+                pos.append(t)
+                flag.append(int(t in sel))
+        t0 = time.perf_counter()
+        oracle.rows(w.q, w.k, w.v, w.g, w.W, seq, head, pos, flag)
+        elapsed += time.perf_counter() - t0
+        done += n_tok
+        n_tok = min(64, n_tok * 2)
+    return {"value": done / elapsed, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{done} random query tokens of the {w.name} workload (all {w.Hq} heads, local + global "
+                      f"where selected, merge), {elapsed:.1f} s of fp64 CPU work"}
+
+
+def run_reference(args, rank, world):
+    """The fp64 CPU oracle as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    from token_level_dynamic_seq_b200 import workloads
+    import oracle
+
+    w = workloads.load(args.workload, seed=0)
+    sel = set(oracle.select(w.g[0], w.ratio).tolist())
+    rng = random.Random(1)
+    per_step = 8  # tokens per step: a bounded sample of the workload
+    times = []
+    for it in range(args.warmup + args.steps):
+        toks = [rng.randrange(w.L) for _ in range(per_step)]
+        seq = [0] * (per_step * w.Hq)
+        head = [h for _ in toks for h in range(w.Hq)]
+        pos = [t for t in toks for _ in range(w.Hq)]
+        flag = [int(t in sel) for t in pos]
+        t0 = time.perf_counter()
+        oracle.rows(w.q, w.k, w.v, w.g, w.W, seq, head, pos, flag)
+        dt = time.perf_counter() - t0
+        if it >= args.warmup:
+            times.append(dt)
+    tot = sum(times)
+    value = per_step * len(times) / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * tot / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "desc": w.recipe, "tokens_per_step": per_step},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"{per_step} random query tokens per step (all {w.Hq} heads, local + global "
+                                   "where selected, merge)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    import token_level_dynamic_seq_b200 as logo
+    from token_level_dynamic_seq_b200 import workloads
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    w = workloads.load(args.workload, seed=rank)
+    q, k, v, g = w.q.to(dev), w.k.to(dev), w.v.to(dev), w.g.to(dev)
+    cu = None if w.cu_seqlens is None else w.cu_seqlens.to(dev)
+    ml = max(w.seqlens)
+    shape = logo.make_shape(q, k, cu, ml)
+    stream = torch.cuda.current_stream(dev)
+    ws = logo.workspace(shape, w.ratio, dev, stream)
+    out = torch.empty_like(q)
+    cap = max(1, logo.selection_capacity(shape, w.ratio, w.seqlens))
+    sel = torch.empty(cap, dtype=torch.int32, device=dev)
+    nseq = len(w.seqlens)
+    cu_sel = torch.empty(nseq + 1, dtype=torch.int32, device=dev)
+    kmax = logo.num_selected(w.ratio, ml)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        logo.select(g, shape, w.ratio, ws, sel, cu_sel, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        logo.local_attn(q, k, v, w.W, ws, cu_seqlens=cu, max_seqlen=ml, out=out, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        logo.global_attn_sparse(q, k, v, g, sel, cu_sel, kmax, out, ws, merge=True, cu_seqlens=cu,
+                                max_seqlen=ml, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    logo.check(ws, stream)
+
+    # useful FLOPs (data-dependent global part from this rank's selection)
+    tot_sel = int(cu_sel[-1].item())
+    sel_pos_sum = int(sel[:tot_sel].to(torch.int64).sum().item()) + tot_sel
+    lp = sum(min(w.W, n) * (min(w.W, n) + 1) // 2 + (n - min(w.W, n)) * min(w.W, n) for n in w.seqlens)
+    fl_local = 4 * w.d * w.Hq * lp
+    fl_global = 4 * w.d * w.Hq * sel_pos_sum
+    tokens = w.tokens
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    t_wall0 = time.perf_counter()
+    for s in range(args.steps):
+        step(evs[s])
+    torch.cuda.synchronize(dev)
+    t_wall = time.perf_counter() - t_wall0
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    logo.check(ws, stream)
+
+    t_total_ms = evs[0][0].elapsed_time(evs[-1][3])
+    per = {"select": [], "local": [], "global": []}
+    for e in evs:
+        per["select"].append(e[0].elapsed_time(e[1]))
+        per["local"].append(e[1].elapsed_time(e[2]))
+        per["global"].append(e[2].elapsed_time(e[3]))
+    avg = {kk: sum(vv) / len(vv) for kk, vv in per.items()}
+    ms_step = t_total_ms / args.steps
+    if world > 1:
+        tt = torch.tensor([ms_step], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_step = float(tt.item())
+
+    # end to end through the public API: pinned host inputs -> forward -> host output
+    pin = [x.pin_memory() for x in (w.q, w.k, w.v, w.g)]
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in pin)
+    d2h = out_host.numel() * out_host.element_size()
+    e2e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e2e_ev[0].record(stream)
+    for _ in range(args.e2e_steps):
+        q.copy_(pin[0], non_blocking=True)
+        k.copy_(pin[1], non_blocking=True)
+        v.copy_(pin[2], non_blocking=True)
+        g.copy_(pin[3], non_blocking=True)
+        logo.forward(q, k, v, g, w.W, w.ratio, ws=ws, cu_seqlens=cu, max_seqlen=ml, out=out, sel_idx=sel,
+                     cu_sel=cu_sel, stream=stream)
+        out_host.copy_(out, non_blocking=True)
+    e2e_ev[1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e2e_ev[0].elapsed_time(e2e_ev[1]) / args.e2e_steps
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    logo.check(ws, stream)
+
+    peak_burst, peak_sust, hbm, peak_src = peaks()
+    dominant = "local" if avg["local"] >= avg["global"] else "global"
+    dom_flops = fl_local if dominant == "local" else fl_global
+    achieved = dom_flops / (avg[dominant] * 1e-3) / 1e12
+    tr = traffic_record()
+    kern_name = {"local": "attn_fwd_kernel<128, 0>", "global": "attn_fwd_kernel<128, 1>"}[dominant]
+    traffic = tr.get(kern_name, {}).get("bytes_per_launch") if isinstance(tr.get(kern_name), dict) else None
+    useful_tflops = (fl_local + fl_global) / (ms_step * 1e-3) / 1e12
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(w)
+        line = {
+            "metric": METRIC,
+            "value": tokens * world / (ms_step * 1e-3),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "desc": w.recipe, "tokens_per_rank": tokens,
+                       "parallelism": f"independent sequences x{world}",
+                       "l2": "inputs larger than L2 (Q+K+V+O = %.0f MB > 126 MB)" % (
+                           (q.numel() + k.numel() + v.numel() + out.numel()) * 2 / 1e6)},
+            "useful_tflops": useful_tflops,
+            "useful_frac_of_bf16_peak": useful_tflops / peak_burst,
+            "kernels_ms": avg,
+            "kernels_tflops": {"local": fl_local / (avg["local"] * 1e-3) / 1e12,
+                               "global": fl_global / (avg["global"] * 1e-3) / 1e12},
+            "useful_flop": {"local": fl_local, "global": fl_global},
+            "roofline": {"kernel": kern_name, "bound": "tensor", "achieved": achieved, "peak": peak_burst,
+                         "unit": "TFLOP/s", "frac": achieved / peak_burst, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16 burst (sustained {peak_sust})"},
+            "e2e": {"value": tokens * world / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clocks,
+            "wall_s_timed": t_wall,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

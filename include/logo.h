@@ -1,0 +1,208 @@
+/*
+ * logo.h -- C ABI of the B200 (sm_100a) library for the forward (prefill)
+ * pass of token-level dynamic local-global attention (LoGo / L2A).
+ *
+ * What the library computes, and where the pages define it:
+ *   - "LoGo: Token-Level Dynamic Local-Global Attention", Abstract: each layer
+ *     has a local and a global branch; every token gets local attention over
+ *     a restricted window; a learned gate gives full-context attention only
+ *     to the tokens that need it; a budget controller keeps a target global
+ *     ratio; query-sparse kernels turn the reduced global work into speed.
+ *   - "Learning When to Attend", "The Architecture of Conditional Attention":
+ *     local attention over a fixed recent window for all tokens, then exact
+ *     attention over the full context for a sparse subset of query tokens
+ *     (about 20% of them).
+ *   - "Local-global attention", Variants, Gemma 2: attention is causal and the
+ *     local kind drops keys more than the window back; Implementation sketch
+ *     notes, "Packed examples (LongT5)": packed examples must be masked per
+ *     example.
+ * Readings of what the pages leave open (fixed here, identical in every entry
+ * point):
+ *   - window: query i attends to key j iff 0 <= i - j < W;
+ *   - budget: k_s = logo_num_selected(ratio, L_s) tokens per sequence, the k_s
+ *     largest gate logits, equal logits broken toward the lower position,
+ *     -0 equal to +0, NaN ranked below -inf; one selection per sequence,
+ *     shared by every head;
+ *   - global branch: exact causal attention over positions 0..i;
+ *   - merge: o_i = local_i + sigmoid(g_i) * global_i on selected rows,
+ *     o_i = local_i elsewhere;
+ *   - GQA: query head h reads key/value head h / (Hq / Hkv);
+ *   - softmax scale: 1/sqrt(d) when `scale` <= 0.
+ *
+ * Conventions shared by every entry point:
+ *   - Ownership: the caller owns every buffer and the stream.  The library
+ *     allocates no memory and never synchronises, except logo_check.  Every
+ *     call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).
+ *   - Device pointers: q, k, v, out, gate, sel_idx, cu_sel, cu_seqlens and ws
+ *     are device (HBM) pointers on the current device, 16-byte aligned,
+ *     contiguous in the stated layout.
+ *   - Element types: q, k, v, out are bf16 (passed as raw 16-bit patterns);
+ *     gate is fp32; indices are int32.
+ *   - Errors: argument problems are reported synchronously as a logo_status
+ *     before anything is launched.  Problems found on the device (a bounded
+ *     wait that ran out) are recorded in a status word inside the workspace;
+ *     logo_check reads it back.
+ *   - Supported shapes: d in {64, 128}; Hq % Hkv == 0; W >= 1;
+ *     0 <= ratio <= 1; sequence lengths < 2^31.
+ */
+#ifndef LOGO_H_
+#define LOGO_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LOGO_API __attribute__((visibility("default")))
+#else
+#define LOGO_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LOGO_OK = 0,
+    LOGO_ERR_INVALID_ARG = 1,    /* a pointer, size or value is out of the supported range */
+    LOGO_ERR_UNSUPPORTED = 2,    /* a shape this build does not implement (e.g. d = 96) */
+    LOGO_ERR_WORKSPACE = 3,      /* workspace missing or smaller than logo_workspace_size() */
+    LOGO_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed (see logo_last_error) */
+    LOGO_ERR_DEVICE_TIMEOUT = 5  /* a kernel's bounded wait ran out (read by logo_check) */
+} logo_status;
+
+/* Raw bf16 bit pattern. */
+typedef uint16_t logo_bf16;
+
+/* A cudaStream_t, passed as an opaque pointer so this header needs no CUDA headers. */
+typedef void *logo_stream_t;
+
+/*
+ * Problem geometry.
+ * Fixed length (cu_seqlens == NULL): B sequences of L tokens; q is
+ *   [B, Hq, L, d], k and v are [B, Hkv, L, d], gate is [B, L], out is
+ *   [B, Hq, L, d]; nseq and max_seqlen are ignored.
+ * Packed varlen (cu_seqlens != NULL): B must be 1 and L is the total token
+ *   count T; sequence s occupies rows cu_seqlens[s] .. cu_seqlens[s+1]-1 of
+ *   every head slab of q/k/v/out and of gate; nseq >= 1 sequences;
+ *   cu_seqlens is a DEVICE int32 array of nseq+1 non-decreasing offsets with
+ *   cu_seqlens[0] == 0 and cu_seqlens[nseq] <= T; max_seqlen must be >= every
+ *   sequence length (it sizes the launch).  No attention crosses a sequence
+ *   boundary; positions, the window and the budget are per sequence.
+ */
+typedef struct {
+    int B, Hq, Hkv, L, d;
+    const int32_t *cu_seqlens;
+    int nseq;
+    int max_seqlen;
+} logo_shape;
+
+/*
+ * Budget count for one sequence ("LoGo", Abstract: target global ratio):
+ * k = ceil(ratio * len), computed in double; a product within 1e-9
+ * (relative, absolute at least 1e-9) of an integer is taken as that integer,
+ * so 0.07 * 100 gives 7, not 8.  Clamped to [0, len].  Host function; never
+ * fails (ratio <= 0 or NaN gives 0).
+ */
+LOGO_API int64_t logo_num_selected(double ratio, int64_t len);
+
+/*
+ * Bytes of device workspace the calls below need for `shape` at `ratio`
+ * (0 if the shape is invalid).  The workspace holds the device status word;
+ * it must be zeroed once with logo_workspace_init before first use and may be
+ * reused by every later call on the same stream.
+ */
+LOGO_API size_t logo_workspace_size(const logo_shape *shape, double ratio);
+
+/* Zero the workspace's status word (asynchronous, on `stream`). */
+LOGO_API logo_status logo_workspace_init(void *ws, size_t ws_bytes, logo_stream_t stream);
+
+/*
+ * Budget rule ("LoGo", Abstract; "Learning When to Attend", "The Architecture
+ * of Conditional Attention"): per sequence, select the k_s =
+ * logo_num_selected(ratio, L_s) positions with the largest gate logits
+ * (ties to the lower position, -0 == +0, NaN below -inf) and write them in
+ * ascending order.
+ *   gate     [B, L] fp32 (device), or [1, T] packed.
+ *   sel_idx  output, int32 (device): the lists of all sequences back to back;
+ *            capacity sum_s k_s (fixed length: B * k with row b at b * k).
+ *            Entries are positions within their sequence (0-based).
+ *   cu_sel   output, int32 [nseq + 1] (device; nseq = B for fixed length):
+ *            cu_sel[s] is where sequence s's list starts, cu_sel[nseq] the total.
+ * Bit-exact: the result is a pure function of the logits' bit patterns.
+ */
+LOGO_API logo_status logo_select(const float *gate, const logo_shape *shape, double ratio, int32_t *sel_idx,
+                        int32_t *cu_sel, void *ws, size_t ws_bytes, logo_stream_t stream);
+
+/*
+ * Local branch for every query ("LoGo", Abstract: local attention over a
+ * restricted window; "Learning When to Attend": a fixed recent window;
+ * "Local-global attention", Gemma 2 variant: causal, keys more than W back
+ * dropped): out[b, h, i] = softmax_j(scale * q_i . k_j) v_j over keys j of
+ * the same sequence with 0 <= i - j < W.  With W >= L this is dense causal
+ * attention.  q, k, v, out as in logo_shape; `scale` <= 0 means 1/sqrt(d).
+ */
+LOGO_API logo_status logo_local_attn(const logo_bf16 *q, const logo_bf16 *k, const logo_bf16 *v,
+                            const logo_shape *shape, int window, float scale, logo_bf16 *out, void *ws,
+                            size_t ws_bytes, logo_stream_t stream);
+
+/*
+ * Query-sparse global branch and gated merge ("Learning When to Attend", "The
+ * Architecture of Conditional Attention": exact attention over the full
+ * context for a sparse subset of query tokens; "LoGo", Abstract: query-sparse
+ * kernels).  For every selected position i of sequence s (from sel_idx /
+ * cu_sel, as written by logo_select) and every query head h:
+ *   global = softmax_j(scale * q_i . k_j) v_j over keys 0..i of sequence s;
+ *   merge != 0: out[i] = out[i] + sigmoid(gate[i]) * global  (out must hold
+ *               the local branch, e.g. from logo_local_attn);
+ *   merge == 0: out[i] = global.
+ * Rows that are not selected are not touched.  `max_selected` is an upper
+ * bound on every sequence's count cu_sel[s+1] - cu_sel[s] (for lists written
+ * by logo_select: logo_num_selected(ratio, longest sequence)); it sizes the
+ * launch, and counts above it are an error the kernel reports in the status
+ * word.  sel_idx entries must be ascending within a sequence and in
+ * [0, L_s).
+ */
+LOGO_API logo_status logo_global_attn_sparse(const logo_bf16 *q, const logo_bf16 *k, const logo_bf16 *v,
+                                    const float *gate, const int32_t *sel_idx, const int32_t *cu_sel,
+                                    const logo_shape *shape, int max_selected, float scale, int merge,
+                                    logo_bf16 *out, void *ws, size_t ws_bytes, logo_stream_t stream);
+
+/*
+ * The whole forward pass: logo_select, logo_local_attn, then
+ * logo_global_attn_sparse with merge, in that order on `stream`.
+ * out receives o; sel_idx / cu_sel receive the selection.
+ */
+LOGO_API logo_status logo_forward(const logo_bf16 *q, const logo_bf16 *k, const logo_bf16 *v, const float *gate,
+                         const logo_shape *shape, int window, double ratio, float scale, logo_bf16 *out,
+                         int32_t *sel_idx, int32_t *cu_sel, void *ws, size_t ws_bytes,
+                         logo_stream_t stream);
+
+/*
+ * Synchronise `stream`, then report: LOGO_ERR_CUDA if a launch or the stream
+ * failed, LOGO_ERR_DEVICE_TIMEOUT if a kernel recorded a bounded wait that ran
+ * out, LOGO_ERR_INVALID_ARG if a kernel recorded an argument it could not
+ * handle, else LOGO_OK.  The only entry point that blocks the host.
+ */
+LOGO_API logo_status logo_check(const void *ws, logo_stream_t stream);
+
+/*
+ * Diagnostic: launch one tiny kernel that waits on a barrier nothing will
+ * complete, with a bound of `limit_us` microseconds; when the bound runs out
+ * it records a timeout in the workspace status word and returns normally
+ * (no trap, no fault).  logo_check then reports LOGO_ERR_DEVICE_TIMEOUT.
+ * Used by the tests of the timeout path.
+ */
+LOGO_API logo_status logo_selftest_timeout(void *ws, size_t ws_bytes, unsigned limit_us, logo_stream_t stream);
+
+/* Static text for a status code. */
+LOGO_API const char *logo_status_string(logo_status status);
+
+/* Details of the last error raised on the calling host thread ("" if none). */
+LOGO_API const char *logo_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOGO_H_ */

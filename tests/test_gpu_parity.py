@@ -1,0 +1,284 @@
+"""Parity of the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Selected indices must match bit for bit.  Outputs must be within max-abs 2e-2
+and relative-L2 5e-3 of the oracle, over everything compared.  Small cases
+compare every element (several 128-row tiles and a ragged tail); the
+full-size workloads, run in the benchmark's launch configuration, compare the
+selection in full and a sample of rows the oracle computes one by one.
+"""
+import math
+import random
+
+import pytest
+import torch
+
+import oracle
+import token_level_dynamic_seq_b200 as logo
+from token_level_dynamic_seq_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-2
+REL_L2 = 5e-3
+
+
+def close(got, ref, what=""):
+    got = got.double().cpu()
+    ref = ref.double().cpu()
+    assert torch.isfinite(got).all(), f"{what}: non-finite output"
+    err = (got - ref).abs().max().item()
+    rel = ((got - ref).norm() / ref.norm().clamp_min(1e-30)).item()
+    assert err <= MAX_ABS and rel <= REL_L2, f"{what}: max-abs {err:.3e}, rel-L2 {rel:.3e}"
+    return err, rel
+
+
+def to_dev(w):
+    cu = None if w.cu_seqlens is None else w.cu_seqlens.cuda()
+    return w.q.cuda(), w.k.cuda(), w.v.cuda(), w.g.cuda(), cu
+
+
+def max_len(w):
+    return max(w.seqlens) if w.seqlens else w.L
+
+
+def sel_lists(sel_idx, cu_sel):
+    cu = cu_sel.cpu().tolist()
+    idx = sel_idx.cpu().tolist()
+    return [idx[cu[s]:cu[s + 1]] for s in range(len(cu) - 1)]
+
+
+def oracle_sel_lists(w):
+    out = []
+    for s, n in enumerate(w.seqlens):
+        if w.cu_seqlens is None:
+            g = w.g[s]
+        else:
+            lo = int(w.cu_seqlens[s])
+            g = w.g[0, lo:lo + n]
+        out.append(oracle.select(g, w.ratio).tolist())
+    return out
+
+
+SMALL = [
+    # name, B, Hq, Hkv, L, d, W, ratio, seqlens
+    ("tiny-like d64 G1", 1, 2, 2, 256, 64, 32, 0.25, None),
+    ("gqa2 ragged", 1, 4, 2, 300, 128, 64, 0.2, None),
+    ("g3 odd group", 2, 3, 1, 513, 64, 200, 0.3, None),
+    ("window1", 1, 2, 2, 1000, 128, 1, 0.1, None),
+    ("dense causal W>=L", 1, 8, 2, 700, 128, 5000, 0.5, None),
+    ("one tile", 1, 2, 1, 129, 128, 128, 0.25, None),
+    ("L=1", 2, 2, 2, 1, 128, 4, 1.0, None),
+    ("gqa4 long window", 1, 8, 2, 1500, 128, 700, 0.2, None),
+    ("varlen", 1, 4, 2, 0, 128, 100, 0.25, [1, 130, 0, 700, 255]),
+    ("varlen d64 g1", 1, 2, 2, 0, 64, 300, 0.35, [513, 3, 1024, 129]),
+]
+
+
+def small_workload(case, seed=0):
+    name, B, Hq, Hkv, L, d, W, ratio, lens = case
+    return workloads.make(B, Hq, Hkv, L, d, W, ratio, seed=seed, qkv_scale=1.0, seqlens=lens, name=name)
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_forward_small_full(case):
+    w = small_workload(case)
+    q, k, v, g, cu = to_dev(w)
+    ml = max_len(w)
+    ws = logo.workspace(logo.make_shape(q, k, cu, ml), w.ratio, q.device)
+    out, sel, cu_sel = logo.forward(q, k, v, g, w.W, w.ratio, ws=ws, cu_seqlens=cu, max_seqlen=ml)
+    logo.check(ws)
+    ref = oracle.forward(w.q, w.k, w.v, w.g, w.W, w.ratio, cu_seqlens=w.cu_seqlens, want_branches=True)
+    assert sel_lists(sel, cu_sel) == oracle_sel_lists(w)
+    assert cu_sel.cpu().tolist() == ref["cu_sel"].tolist()
+    # local branch alone
+    loc = logo.local_attn(q, k, v, w.W, ws, cu_seqlens=cu, max_seqlen=ml)
+    logo.check(ws)
+    if w.cu_seqlens is None:
+        close(loc, ref["local"], "local")
+        close(out, ref["out"], "merged")
+    else:  # rows outside every sequence are not written
+        T = int(w.cu_seqlens[-1])
+        close(loc[:, :, :T], ref["local"][:, :, :T], "local")
+        close(out[:, :, :T], ref["out"][:, :, :T], "merged")
+    # raw global branch on the selected rows (merge = 0), other rows untouched
+    sentinel = torch.full_like(q, 7.0)
+    kmax = logo.num_selected(w.ratio, ml)
+    logo.global_attn_sparse(q, k, v, g, sel, cu_sel, kmax, sentinel, ws, merge=False, cu_seqlens=cu,
+                            max_seqlen=ml)
+    logo.check(ws)
+    rows = []
+    for s, lst in enumerate(sel_lists(sel, cu_sel)):
+        base = 0 if w.cu_seqlens is None else int(w.cu_seqlens[s])
+        b = s if w.cu_seqlens is None else 0
+        rows += [(b, base + i) for i in lst]
+    if rows:
+        bi = torch.tensor([r[0] for r in rows])
+        ti = torch.tensor([r[1] for r in rows])
+        got = sentinel.cpu()[bi, :, ti]
+        close(got, ref["global"][bi, :, ti], "global")
+        mask = torch.ones(sentinel.shape[0], sentinel.shape[2], dtype=torch.bool)
+        mask[bi, ti] = False
+        untouched = sentinel.cpu().permute(0, 2, 1, 3)[mask]
+        assert (untouched == 7.0).all()
+
+
+def test_forward_is_deterministic():
+    w = small_workload(SMALL[7], seed=3)
+    q, k, v, g, cu = to_dev(w)
+    ws = logo.workspace(logo.make_shape(q, k), w.ratio, q.device)
+    o1, s1, c1 = logo.forward(q, k, v, g, w.W, w.ratio, ws=ws)
+    o2, s2, c2 = logo.forward(q, k, v, g, w.W, w.ratio, ws=ws)
+    logo.check(ws)
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(s1, s2) and torch.equal(c1, c2)
+
+
+def test_no_writes_outside_output():
+    w = small_workload(SMALL[2], seed=5)
+    q, k, v, g, cu = to_dev(w)
+    n = q.numel()
+    buf = torch.full((n + 2 * 4096,), -3.0, dtype=torch.bfloat16, device="cuda")
+    out = buf[4096:4096 + n].view_as(q)
+    ws = logo.workspace(logo.make_shape(q, k), w.ratio, q.device)
+    logo.forward(q, k, v, g, w.W, w.ratio, ws=ws, out=out)
+    logo.check(ws)
+    assert (buf[:4096] == -3.0).all() and (buf[4096 + n:] == -3.0).all()
+
+
+# --------------------------------------------------------------------------
+# selection: bit-exact on adversarial logits
+# --------------------------------------------------------------------------
+
+def _select_gpu(g, ratio):
+    L = g.numel()
+    gd = g.view(1, L).cuda()
+    sh = logo.Shape(1, 1, 1, L, 128, None, 1, L)
+    ws = logo.workspace(sh, ratio, gd.device)
+    sel, cu_sel = logo.select(gd, sh, ratio, ws)
+    logo.check(ws)
+    return sel[:int(cu_sel[1])].cpu().tolist()
+
+
+def test_select_golden_cases():
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "select_cases.txt")
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        ratio, logits, expect = [x.strip() for x in line.split("|")]
+        g = torch.tensor([float(t) for t in logits.split(",")], dtype=torch.float32)
+        want = [int(t) for t in expect.split(",")] if expect else []
+        assert _select_gpu(g, float(ratio)) == want, line
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_select_random_ties_specials(seed):
+    rng = random.Random(seed)
+    n = rng.choice([5, 1000, 4097, 65536, 131072])
+    gen = torch.Generator().manual_seed(seed)
+    g = torch.randn(n, generator=gen)
+    if seed % 2 == 0:
+        g = (g * 4).round() / 4  # heavy ties
+    specials = torch.tensor([0.0, -0.0, float("inf"), float("-inf"), float("nan"), 1e-45, -1e-45])
+    idx = torch.randint(0, n, (max(1, n // 50),), generator=gen)
+    g[idx] = specials[torch.randint(0, len(specials), (idx.numel(),), generator=gen)]
+    for ratio in (0.0, 0.05, 0.2, 0.5, 0.999, 1.0):
+        assert _select_gpu(g, ratio) == oracle.select(g, ratio).tolist()
+
+
+# --------------------------------------------------------------------------
+# the named workloads at full size, in the benchmark's launch configuration
+# --------------------------------------------------------------------------
+
+def sampled_rows(w, sel_lists_, n_random=192, n_sel=96, seed=0):
+    rng = random.Random(seed)
+    rows = []
+    nonempty = [s for s, n in enumerate(w.seqlens) if n > 0]
+    for _ in range(n_random):
+        s = rng.choice(nonempty)
+        rows.append((s, rng.randrange(w.Hq), rng.randrange(w.seqlens[s])))
+    with_sel = [s for s in nonempty if sel_lists_[s]]
+    for _ in range(n_sel if with_sel else 0):
+        s = rng.choice(with_sel)
+        rows.append((s, rng.randrange(w.Hq), rng.choice(sel_lists_[s])))
+    # the first and last rows of a sequence (tile and window edges)
+    s = nonempty[-1]
+    rows += [(s, 0, 0), (s, w.Hq - 1, w.seqlens[s] - 1)]
+    return rows
+
+
+def check_sampled(w, out, sel_lists_, seed=0):
+    rows = sampled_rows(w, sel_lists_, seed=seed)
+    sets = [set(x) for x in sel_lists_]
+    loc, glo, ref = oracle.rows(w.q, w.k, w.v, w.g, w.W, [r[0] for r in rows], [r[1] for r in rows],
+                                [r[2] for r in rows], [int(r[2] in sets[r[0]]) for r in rows],
+                                cu_seqlens=w.cu_seqlens)
+    outc = out.cpu()
+    got = []
+    for s, h, i in rows:
+        if w.cu_seqlens is None:
+            got.append(outc[s, h, i])
+        else:
+            got.append(outc[0, h, int(w.cu_seqlens[s]) + i])
+    return close(torch.stack(got), ref, f"{w.name} sampled")
+
+
+def run_full(w):
+    q, k, v, g, cu = to_dev(w)
+    ml = max_len(w)
+    ws = logo.workspace(logo.make_shape(q, k, cu, ml), w.ratio, q.device)
+    out, sel, cu_sel = logo.forward(q, k, v, g, w.W, w.ratio, ws=ws, cu_seqlens=cu, max_seqlen=ml)
+    logo.check(ws)
+    return out, sel_lists(sel, cu_sel), cu_sel
+
+
+@pytest.mark.parametrize("name", ["tiny", "c4k"])
+def test_named_small_full(name):
+    w = workloads.load(name)
+    out, lists, cu_sel = run_full(w)
+    ref = oracle.forward(w.q, w.k, w.v, w.g, w.W, w.ratio)
+    assert lists == oracle_sel_lists(w)
+    assert cu_sel.cpu().tolist() == ref["cu_sel"].tolist()
+    close(out, ref["out"], name)
+
+
+@pytest.mark.parametrize("name", ["c32k", "varlen"])
+def test_named_large_sampled(name):
+    w = workloads.load(name)
+    out, lists, _ = run_full(w)
+    assert lists == oracle_sel_lists(w)
+    check_sampled(w, out, lists)
+
+
+def test_c128k_ratio_sweep_sampled():
+    base = workloads.load("c128k_r0.2")
+    for r in workloads.RATIO_SWEEP_128K:
+        base.ratio = r
+        base.name = f"c128k_r{r:g}"
+        out, lists, _ = run_full(base)
+        assert lists == oracle_sel_lists(base)
+        check_sampled(base, out, lists, seed=int(r * 100))
+        del out
+        torch.cuda.empty_cache()
+
+
+# --------------------------------------------------------------------------
+# bounded waits: a wait that runs out reports an error and the context stays usable
+# --------------------------------------------------------------------------
+
+def test_timeout_is_reported_and_context_survives():
+    sh = logo.Shape(1, 2, 2, 256, 64, None, 1, 256)
+    ws = logo.workspace(sh, 0.25, torch.device("cuda"))
+    logo.selftest_timeout(ws, limit_us=2000)
+    with pytest.raises(logo.LogoError) as e:
+        logo.check(ws)
+    assert e.value.status == 5
+    # clear and run a real call on the same context
+    ws2 = logo.workspace(sh, 0.25, torch.device("cuda"))
+    w = workloads.load("tiny")
+    q, k, v, g, _ = to_dev(w)
+    out, sel, cu_sel = logo.forward(q, k, v, g, w.W, w.ratio, ws=ws2)
+    logo.check(ws2)
+    ref = oracle.forward(w.q, w.k, w.v, w.g, w.W, w.ratio)
+    close(out, ref["out"], "after timeout")

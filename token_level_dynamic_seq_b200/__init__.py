@@ -1,1 +1,224 @@
-"""B200-native token-level dynamic local-global attention (placeholder, binding follows)."""
+"""B200-native (sm_100a) forward pass of token-level dynamic local-global attention.
+
+Method (page titles and sections): "LoGo: Token-Level Dynamic Local-Global
+Attention", Abstract; "Learning When to Attend", "The Architecture of
+Conditional Attention".  Every query token gets causal sliding-window
+attention over the previous W keys; a per-sequence budget picks the
+ceil(ratio * L) tokens with the largest gate logits (ties to the lower
+position); those tokens also get exact full-causal attention, merged as
+``local + sigmoid(g) * global``.
+
+This module is a thin ctypes binding over the C ABI in ``include/logo.h``
+(``liblogo.so``): it only marshals torch CUDA tensors (device memory, the
+current stream) into the C calls.  Every step of the computation runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback, and a missing
+library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblogo.so")
+CSRC = os.path.join(_HERE, "csrc")
+
+LOGO_OK = 0
+_STATUS = {0: "LOGO_OK", 1: "LOGO_ERR_INVALID_ARG", 2: "LOGO_ERR_UNSUPPORTED", 3: "LOGO_ERR_WORKSPACE",
+           4: "LOGO_ERR_CUDA", 5: "LOGO_ERR_DEVICE_TIMEOUT"}
+
+EXPORTED = ("logo_num_selected", "logo_workspace_size", "logo_workspace_init", "logo_select",
+            "logo_local_attn", "logo_global_attn_sparse", "logo_forward", "logo_check",
+            "logo_selftest_timeout", "logo_status_string", "logo_last_error")
+
+
+class LogoError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        super().__init__(f"{_STATUS.get(status, status)}: {message}")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("L", ctypes.c_int),
+                ("d", ctypes.c_int), ("cu_seqlens", ctypes.c_void_p), ("nseq", ctypes.c_int),
+                ("max_seqlen", ctypes.c_int)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load_library(path: str | None = None):
+    """Load liblogo.so (built by ``make -C token_level_dynamic_seq_b200/csrc``); raise if absent."""
+    global _lib
+    with _lock:
+        if _lib is not None and path is None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(f"CUDA library {p} is missing: build it with `make -C {CSRC}` "
+                               "(or __graft_entry__.build()); there is no fallback")
+        lib = ctypes.CDLL(p)
+        vp, i32, i64, dbl, flt, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double,
+                                      ctypes.c_float, ctypes.c_size_t)
+        sp = ctypes.POINTER(Shape)
+        sig = {
+            "logo_num_selected": ([dbl, i64], i64),
+            "logo_workspace_size": ([sp, dbl], sz),
+            "logo_workspace_init": ([vp, sz, vp], i32),
+            "logo_select": ([vp, sp, dbl, vp, vp, vp, sz, vp], i32),
+            "logo_local_attn": ([vp, vp, vp, sp, i32, flt, vp, vp, sz, vp], i32),
+            "logo_global_attn_sparse": ([vp, vp, vp, vp, vp, vp, sp, i32, flt, i32, vp, vp, sz, vp], i32),
+            "logo_forward": ([vp, vp, vp, vp, sp, i32, dbl, flt, vp, vp, vp, vp, sz, vp], i32),
+            "logo_check": ([vp, vp], i32),
+            "logo_selftest_timeout": ([vp, sz, ctypes.c_uint, vp], i32),
+            "logo_status_string": ([i32], ctypes.c_char_p),
+            "logo_last_error": ([], ctypes.c_char_p),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(lib, name)
+            f.argtypes = args
+            f.restype = res
+        if path is None:
+            _lib = lib
+        return lib
+
+
+def _raise(status: int):
+    if status != LOGO_OK:
+        msg = load_library().logo_last_error().decode()
+        raise LogoError(status, msg)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _bits(x: torch.Tensor) -> torch.Tensor:
+    if x.dtype != torch.bfloat16:
+        raise TypeError(f"expected bf16, got {x.dtype}")
+    if not x.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not x.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return x
+
+
+def make_shape(q: torch.Tensor, k: torch.Tensor, cu_seqlens=None, max_seqlen=None) -> Shape:
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    if cu_seqlens is None:
+        return Shape(B, Hq, Hkv, L, d, None, B, L)
+    nseq = cu_seqlens.numel() - 1
+    if max_seqlen is None:
+        raise ValueError("max_seqlen is required with cu_seqlens (the library never reads device data on the host)")
+    return Shape(B, Hq, Hkv, L, d, cu_seqlens.data_ptr(), nseq, int(max_seqlen))
+
+
+def num_selected(ratio: float, length: int) -> int:
+    return int(load_library().logo_num_selected(float(ratio), int(length)))
+
+
+def workspace(shape: Shape, ratio: float, device, stream=None) -> torch.Tensor:
+    lib = load_library()
+    n = lib.logo_workspace_size(ctypes.byref(shape), float(ratio))
+    if n == 0:
+        _raise(1)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    _raise(lib.logo_workspace_init(_ptr(ws), ws.numel(), _stream(stream)))
+    return ws
+
+
+def check(ws: torch.Tensor, stream=None):
+    """Synchronise the stream and raise if a kernel recorded an error."""
+    _raise(load_library().logo_check(_ptr(ws), _stream(stream)))
+
+
+def selection_capacity(shape: Shape, ratio: float, seqlens=None) -> int:
+    if shape.cu_seqlens is None or not shape.cu_seqlens:
+        return shape.B * num_selected(ratio, shape.L)
+    if seqlens is None:
+        # upper bound without reading device data: every sequence at max_seqlen, capped by T
+        return min(shape.L, shape.nseq * num_selected(ratio, shape.max_seqlen))
+    return sum(num_selected(ratio, n) for n in seqlens)
+
+
+def select(gate: torch.Tensor, shape: Shape, ratio: float, ws: torch.Tensor, sel_idx=None, cu_sel=None,
+           stream=None):
+    lib = load_library()
+    nseq = shape.nseq if shape.cu_seqlens else shape.B
+    if sel_idx is None:
+        sel_idx = torch.empty(max(1, selection_capacity(shape, ratio)), dtype=torch.int32, device=gate.device)
+    if cu_sel is None:
+        cu_sel = torch.empty(nseq + 1, dtype=torch.int32, device=gate.device)
+    _raise(lib.logo_select(_ptr(gate), ctypes.byref(shape), float(ratio), _ptr(sel_idx), _ptr(cu_sel), _ptr(ws),
+                           ws.numel(), _stream(stream)))
+    return sel_idx, cu_sel
+
+
+def local_attn(q, k, v, window: int, ws: torch.Tensor, scale: float = 0.0, cu_seqlens=None, max_seqlen=None,
+               out=None, stream=None):
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    shape = make_shape(q, k, cu_seqlens, max_seqlen)
+    if out is None:
+        out = torch.empty_like(q)
+    _raise(load_library().logo_local_attn(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(shape), int(window),
+                                          float(scale), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def global_attn_sparse(q, k, v, gate, sel_idx, cu_sel, max_selected: int, out, ws: torch.Tensor,
+                       scale: float = 0.0, merge: bool = True, cu_seqlens=None, max_seqlen=None, stream=None):
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    shape = make_shape(q, k, cu_seqlens, max_seqlen)
+    _raise(load_library().logo_global_attn_sparse(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(sel_idx), _ptr(cu_sel), ctypes.byref(shape),
+        int(max_selected), float(scale), 1 if merge else 0, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def forward(q, k, v, gate, window: int, ratio: float, ws: torch.Tensor | None = None, scale: float = 0.0,
+            cu_seqlens=None, max_seqlen=None, out=None, sel_idx=None, cu_sel=None, stream=None):
+    """The whole forward pass; returns (out, sel_idx, cu_sel)."""
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    shape = make_shape(q, k, cu_seqlens, max_seqlen)
+    if ws is None:
+        ws = workspace(shape, ratio, q.device, stream)
+    if out is None:
+        out = torch.empty_like(q)
+    nseq = shape.nseq if cu_seqlens is not None else shape.B
+    if sel_idx is None:
+        sel_idx = torch.empty(max(1, selection_capacity(shape, ratio)), dtype=torch.int32, device=q.device)
+    if cu_sel is None:
+        cu_sel = torch.empty(nseq + 1, dtype=torch.int32, device=q.device)
+    _raise(load_library().logo_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(gate), ctypes.byref(shape), int(window),
+                                       float(ratio), float(scale), _ptr(out), _ptr(sel_idx), _ptr(cu_sel),
+                                       _ptr(ws), ws.numel(), _stream(stream)))
+    return out, sel_idx, cu_sel
+
+
+def selftest_timeout(ws: torch.Tensor, limit_us: int = 1000, stream=None):
+    _raise(load_library().logo_selftest_timeout(_ptr(ws), ws.numel(), int(limit_us), _stream(stream)))
+
+
+def useful_flops(d: int, Hq: int, seqlens, window: int, sel_positions) -> tuple[int, int]:
+    """Useful FLOPs of one forward pass: (local, global).
+
+    local = 4 d Hq sum_s sum_{i < L_s} min(i + 1, W); global = 4 d Hq sum_{i selected} (i + 1).
+    """
+    lp = 0
+    for n in seqlens:
+        n = int(n)
+        w = min(int(window), n)
+        # sum_{i<n} min(i+1, w) = w(w+1)/2 + (n - w) w
+        lp += w * (w + 1) // 2 + (n - w) * w
+    sp = int(sum(int(p) + 1 for p in sel_positions))
+    return 4 * d * Hq * lp, 4 * d * Hq * sp

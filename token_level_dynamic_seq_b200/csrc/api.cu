@@ -1,0 +1,356 @@
+// C ABI entry points (declared in include/logo.h): argument validation, TMA
+// descriptor set-up and kernel launches.  No allocation, no synchronisation
+// except in logo_check.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.cuh"
+#include "logo.h"
+
+namespace {
+
+using logo::AttnParams;
+
+thread_local char g_last_error[512] = "";
+
+logo_status fail(logo_status s, const char* fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+logo_status cuda_fail(cudaError_t e, const char* what)
+{
+    return fail(LOGO_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Workspace layout: a 256-byte header whose first word is the device status.
+constexpr size_t kWsHeaderBytes = 256;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Geometry after validation.
+struct Geo {
+    int B, Hq, Hkv, L, d, G, nseq, max_len;
+    const int32_t* cu;
+};
+
+logo_status check_shape(const logo_shape* sh, Geo& g)
+{
+    if (!sh) return fail(LOGO_ERR_INVALID_ARG, "shape is NULL");
+    g.B = sh->B;
+    g.Hq = sh->Hq;
+    g.Hkv = sh->Hkv;
+    g.L = sh->L;
+    g.d = sh->d;
+    g.cu = sh->cu_seqlens;
+    if (g.d != 64 && g.d != 128) return fail(LOGO_ERR_UNSUPPORTED, "head dim d=%d (supported: 64, 128)", g.d);
+    if (g.B < 1 || g.Hq < 1 || g.Hkv < 1 || g.L < 0)
+        return fail(LOGO_ERR_INVALID_ARG, "B=%d Hq=%d Hkv=%d L=%d out of range", g.B, g.Hq, g.Hkv, g.L);
+    if (g.Hq % g.Hkv != 0) return fail(LOGO_ERR_INVALID_ARG, "Hq=%d is not a multiple of Hkv=%d", g.Hq, g.Hkv);
+    g.G = g.Hq / g.Hkv;
+    if (g.cu) {
+        if (g.B != 1) return fail(LOGO_ERR_INVALID_ARG, "packed varlen layout needs B == 1 (got %d)", g.B);
+        if (!aligned16(g.cu) && (reinterpret_cast<uintptr_t>(g.cu) & 3u))
+            return fail(LOGO_ERR_INVALID_ARG, "cu_seqlens is not 4-byte aligned");
+        if (sh->nseq < 1) return fail(LOGO_ERR_INVALID_ARG, "nseq=%d must be >= 1", sh->nseq);
+        if (sh->max_seqlen < 0 || sh->max_seqlen > g.L)
+            return fail(LOGO_ERR_INVALID_ARG, "max_seqlen=%d outside [0, L=%d]", sh->max_seqlen, g.L);
+        g.nseq = sh->nseq;
+        g.max_len = sh->max_seqlen;
+    } else {
+        g.nseq = g.B;
+        g.max_len = g.L;
+    }
+    const double rows = (double)g.B * (double)(g.Hq > g.Hkv ? g.Hq : g.Hkv) * (double)g.L;
+    if (rows >= 2147483647.0) return fail(LOGO_ERR_UNSUPPORTED, "B*H*L=%.0f rows exceeds 2^31-1", rows);
+    return LOGO_OK;
+}
+
+logo_status check_ptr(const void* p, const char* name)
+{
+    if (!p) return fail(LOGO_ERR_INVALID_ARG, "%s is NULL", name);
+    if (!aligned16(p)) return fail(LOGO_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+    return LOGO_OK;
+}
+
+logo_status check_ws(void* ws, size_t ws_bytes)
+{
+    if (!ws || ws_bytes < kWsHeaderBytes || !aligned16(ws))
+        return fail(LOGO_ERR_WORKSPACE, "workspace %p of %zu bytes (need >= %zu, 16-byte aligned)", ws, ws_bytes,
+                    kWsHeaderBytes);
+    return LOGO_OK;
+}
+
+logo_status check_ratio(double ratio)
+{
+    if (!(ratio >= 0.0 && ratio <= 1.0)) return fail(LOGO_ERR_INVALID_ARG, "ratio=%g outside [0, 1]", ratio);
+    return LOGO_OK;
+}
+
+logo_status resolve_scale(float scale, int d, float& scale_log2)
+{
+    if (std::isnan(scale) || std::isinf(scale)) return fail(LOGO_ERR_INVALID_ARG, "scale is not finite");
+    const double s = scale > 0.f ? (double)scale : 1.0 / std::sqrt((double)d);
+    scale_log2 = (float)(s * 1.4426950408889634);  // log2(e)
+    return LOGO_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn(logo_status& st)
+{
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    static cudaError_t err = cudaSuccess;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        err = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q);
+        if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    st = fn ? LOGO_OK
+            : fail(LOGO_ERR_CUDA, "cuTensorMapEncodeTiled unavailable: %s", cudaGetErrorString(err));
+    return fn;
+}
+
+// 3-D bf16 view [slabs][rows][d] with a box of 64 x 128 x 1 and the 128B swizzle.
+logo_status make_map(CUtensorMap* map, const void* base, int d, int rows, int slabs)
+{
+    logo_status st;
+    EncodeTiledFn fn = encode_fn(st);
+    if (!fn) return st;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)(rows > 0 ? rows : 1), (cuuint64_t)slabs};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * (cuuint64_t)(rows > 0 ? rows : 1)};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(LOGO_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return LOGO_OK;
+}
+
+void base_params(AttnParams& p, const Geo& g, const void* q, const void* k, const void* v, void* out,
+                 float scale_log2, void* ws)
+{
+    memset(&p, 0, sizeof p);
+    p.q = static_cast<const uint16_t*>(q);
+    p.out = static_cast<uint16_t*>(out);
+    p.cu_seqlens = g.cu;
+    p.status = static_cast<uint32_t*>(ws);
+    p.Hq = g.Hq;
+    p.Hkv = g.Hkv;
+    p.G = g.G;
+    p.L = g.L;
+    p.nseq = g.nseq;
+    p.pair_heads = (g.G % 2 == 0) ? 1 : 0;
+    p.scale_log2 = scale_log2;
+    p.timeout_ns = 1000000000ull;  // 1 s per wait: far above any legitimate stall
+    (void)k;
+    (void)v;
+}
+
+logo_status launch_local(const Geo& g, const void* q, const void* k, const void* v, int window, float scale_log2,
+                         void* out, void* ws, cudaStream_t stream)
+{
+    if (g.L == 0 || g.max_len == 0) return LOGO_OK;
+    AttnParams p;
+    base_params(p, g, q, k, v, out, scale_log2, ws);
+    p.window = window < g.max_len ? window : (g.max_len > 0 ? g.max_len : 1);
+    logo_status st;
+    if ((st = make_map(&p.tm_q, q, g.d, g.L, g.B * g.Hq)) != LOGO_OK) return st;
+    if ((st = make_map(&p.tm_k, k, g.d, g.L, g.B * g.Hkv)) != LOGO_OK) return st;
+    if ((st = make_map(&p.tm_v, v, g.d, g.L, g.B * g.Hkv)) != LOGO_OK) return st;
+    cudaError_t e = logo::launch_attn(logo::kModeLocal, g.d, p, g.max_len, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "local attention launch");
+    return LOGO_OK;
+}
+
+logo_status launch_global(const Geo& g, const void* q, const void* k, const void* v, const float* gate,
+                          const int32_t* sel_idx, const int32_t* cu_sel, int max_selected, float scale_log2,
+                          int merge, void* out, void* ws, cudaStream_t stream)
+{
+    if (g.L == 0 || g.max_len == 0 || max_selected == 0) return LOGO_OK;
+    AttnParams p;
+    base_params(p, g, q, k, v, out, scale_log2, ws);
+    p.gate = gate;
+    p.sel_idx = sel_idx;
+    p.cu_sel = cu_sel;
+    p.max_selected = max_selected;
+    p.merge = merge ? 1 : 0;
+    p.window = g.max_len;
+    logo_status st;
+    if ((st = make_map(&p.tm_k, k, g.d, g.L, g.B * g.Hkv)) != LOGO_OK) return st;
+    if ((st = make_map(&p.tm_v, v, g.d, g.L, g.B * g.Hkv)) != LOGO_OK) return st;
+    cudaError_t e = logo::launch_attn(logo::kModeGlobal, g.d, p, g.max_len, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "global attention launch");
+    return LOGO_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t logo_num_selected(double ratio, int64_t len) { return logo::budget_count(ratio, len); }
+
+size_t logo_workspace_size(const logo_shape* shape, double ratio)
+{
+    Geo g;
+    if (check_shape(shape, g) != LOGO_OK || check_ratio(ratio) != LOGO_OK) return 0;
+    return kWsHeaderBytes;
+}
+
+logo_status logo_workspace_init(void* ws, size_t ws_bytes, logo_stream_t stream)
+{
+    logo_status st = check_ws(ws, ws_bytes);
+    if (st != LOGO_OK) return st;
+    cudaError_t e = cudaMemsetAsync(ws, 0, kWsHeaderBytes, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? LOGO_OK : cuda_fail(e, "workspace init");
+}
+
+logo_status logo_select(const float* gate, const logo_shape* shape, double ratio, int32_t* sel_idx, int32_t* cu_sel,
+                        void* ws, size_t ws_bytes, logo_stream_t stream)
+{
+    Geo g;
+    logo_status st;
+    if ((st = check_shape(shape, g)) != LOGO_OK) return st;
+    if ((st = check_ratio(ratio)) != LOGO_OK) return st;
+    if ((st = check_ws(ws, ws_bytes)) != LOGO_OK) return st;
+    if ((st = check_ptr(cu_sel, "cu_sel")) != LOGO_OK) return st;
+    if (g.L > 0 && (st = check_ptr(gate, "gate")) != LOGO_OK) return st;
+    if (g.L > 0 && logo::budget_count(ratio, g.max_len) > 0 && (st = check_ptr(sel_idx, "sel_idx")) != LOGO_OK)
+        return st;
+    cudaError_t e;
+    if (g.L == 0 && !g.cu) {
+        e = cudaMemsetAsync(cu_sel, 0, sizeof(int32_t) * (size_t)(g.nseq + 1), static_cast<cudaStream_t>(stream));
+    } else {
+        e = logo::launch_select(gate, g.cu, g.nseq, g.L, ratio, sel_idx, cu_sel, static_cast<cudaStream_t>(stream));
+    }
+    return e == cudaSuccess ? LOGO_OK : cuda_fail(e, "select launch");
+}
+
+logo_status logo_local_attn(const logo_bf16* q, const logo_bf16* k, const logo_bf16* v, const logo_shape* shape,
+                            int window, float scale, logo_bf16* out, void* ws, size_t ws_bytes, logo_stream_t stream)
+{
+    Geo g;
+    logo_status st;
+    float sl2;
+    if ((st = check_shape(shape, g)) != LOGO_OK) return st;
+    if (window < 1) return fail(LOGO_ERR_INVALID_ARG, "window=%d must be >= 1", window);
+    if ((st = resolve_scale(scale, g.d, sl2)) != LOGO_OK) return st;
+    if ((st = check_ws(ws, ws_bytes)) != LOGO_OK) return st;
+    if (g.L > 0) {
+        if ((st = check_ptr(q, "q")) != LOGO_OK || (st = check_ptr(k, "k")) != LOGO_OK ||
+            (st = check_ptr(v, "v")) != LOGO_OK || (st = check_ptr(out, "out")) != LOGO_OK)
+            return st;
+    }
+    return launch_local(g, q, k, v, window, sl2, out, ws, static_cast<cudaStream_t>(stream));
+}
+
+logo_status logo_global_attn_sparse(const logo_bf16* q, const logo_bf16* k, const logo_bf16* v, const float* gate,
+                                    const int32_t* sel_idx, const int32_t* cu_sel, const logo_shape* shape,
+                                    int max_selected, float scale, int merge, logo_bf16* out, void* ws,
+                                    size_t ws_bytes, logo_stream_t stream)
+{
+    Geo g;
+    logo_status st;
+    float sl2;
+    if ((st = check_shape(shape, g)) != LOGO_OK) return st;
+    if ((st = resolve_scale(scale, g.d, sl2)) != LOGO_OK) return st;
+    if ((st = check_ws(ws, ws_bytes)) != LOGO_OK) return st;
+    if (max_selected < 0 || max_selected > g.max_len)
+        return fail(LOGO_ERR_INVALID_ARG, "max_selected=%d outside [0, %d]", max_selected, g.max_len);
+    if (g.L > 0 && max_selected > 0) {
+        if ((st = check_ptr(q, "q")) != LOGO_OK || (st = check_ptr(k, "k")) != LOGO_OK ||
+            (st = check_ptr(v, "v")) != LOGO_OK || (st = check_ptr(out, "out")) != LOGO_OK ||
+            (st = check_ptr(sel_idx, "sel_idx")) != LOGO_OK || (st = check_ptr(cu_sel, "cu_sel")) != LOGO_OK)
+            return st;
+        if (merge && (st = check_ptr(gate, "gate")) != LOGO_OK) return st;
+    }
+    return launch_global(g, q, k, v, gate, sel_idx, cu_sel, max_selected, sl2, merge, out, ws,
+                         static_cast<cudaStream_t>(stream));
+}
+
+logo_status logo_forward(const logo_bf16* q, const logo_bf16* k, const logo_bf16* v, const float* gate,
+                         const logo_shape* shape, int window, double ratio, float scale, logo_bf16* out,
+                         int32_t* sel_idx, int32_t* cu_sel, void* ws, size_t ws_bytes, logo_stream_t stream)
+{
+    Geo g;
+    logo_status st;
+    float sl2;
+    if ((st = check_shape(shape, g)) != LOGO_OK) return st;
+    if ((st = check_ratio(ratio)) != LOGO_OK) return st;
+    if (window < 1) return fail(LOGO_ERR_INVALID_ARG, "window=%d must be >= 1", window);
+    if ((st = resolve_scale(scale, g.d, sl2)) != LOGO_OK) return st;
+    if ((st = check_ws(ws, ws_bytes)) != LOGO_OK) return st;
+    if ((st = check_ptr(cu_sel, "cu_sel")) != LOGO_OK) return st;
+    const int max_sel = (int)logo::budget_count(ratio, g.max_len);
+    if (g.L > 0) {
+        if ((st = check_ptr(q, "q")) != LOGO_OK || (st = check_ptr(k, "k")) != LOGO_OK ||
+            (st = check_ptr(v, "v")) != LOGO_OK || (st = check_ptr(out, "out")) != LOGO_OK ||
+            (st = check_ptr(gate, "gate")) != LOGO_OK)
+            return st;
+        if (max_sel > 0 && (st = check_ptr(sel_idx, "sel_idx")) != LOGO_OK) return st;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = logo_select(gate, shape, ratio, sel_idx, cu_sel, ws, ws_bytes, stream)) != LOGO_OK) return st;
+    if ((st = launch_local(g, q, k, v, window, sl2, out, ws, s)) != LOGO_OK) return st;
+    return launch_global(g, q, k, v, gate, sel_idx, cu_sel, max_sel, sl2, 1, out, ws, s);
+}
+
+logo_status logo_check(const void* ws, logo_stream_t stream)
+{
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "pending launch error");
+    if (!ws) return fail(LOGO_ERR_WORKSPACE, "workspace is NULL");
+    uint32_t status = 0;
+    e = cudaMemcpy(&status, ws, sizeof status, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "status read");
+    if (status & logo::kStatusTimeout)
+        return fail(LOGO_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait ran out (status 0x%x)", status);
+    if (status & logo::kStatusBadArgument)
+        return fail(LOGO_ERR_INVALID_ARG, "a kernel met an argument it cannot handle (status 0x%x)", status);
+    return LOGO_OK;
+}
+
+logo_status logo_selftest_timeout(void* ws, size_t ws_bytes, unsigned limit_us, logo_stream_t stream)
+{
+    logo_status st = check_ws(ws, ws_bytes);
+    if (st != LOGO_OK) return st;
+    if (limit_us == 0 || limit_us > 10000000u)
+        return fail(LOGO_ERR_INVALID_ARG, "limit_us=%u outside [1, 10^7]", limit_us);
+    cudaError_t e = logo::launch_timeout_probe(static_cast<uint32_t*>(ws), 1000ull * limit_us,
+                                               static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? LOGO_OK : cuda_fail(e, "timeout probe launch");
+}
+
+const char* logo_status_string(logo_status s)
+{
+    switch (s) {
+        case LOGO_OK: return "LOGO_OK";
+        case LOGO_ERR_INVALID_ARG: return "LOGO_ERR_INVALID_ARG";
+        case LOGO_ERR_UNSUPPORTED: return "LOGO_ERR_UNSUPPORTED";
+        case LOGO_ERR_WORKSPACE: return "LOGO_ERR_WORKSPACE";
+        case LOGO_ERR_CUDA: return "LOGO_ERR_CUDA";
+        case LOGO_ERR_DEVICE_TIMEOUT: return "LOGO_ERR_DEVICE_TIMEOUT";
+    }
+    return "LOGO_ERR_UNKNOWN";
+}
+
+const char* logo_last_error(void) { return g_last_error; }
+
+}  // extern "C"

@@ -1,0 +1,576 @@
+// Local (sliding-window) and query-sparse global attention forward kernels
+// for sm_100a, with the gated merge fused into the global kernel's epilogue.
+//
+// Method sources (page titles and sections):
+//  * "LoGo: Token-Level Dynamic Local-Global Attention", Abstract: all tokens
+//    get local attention over a restricted window; a gate activates
+//    full-context attention only for some tokens; query-sparse kernels turn
+//    the reduced global work into speed.
+//  * "Learning When to Attend", "The Architecture of Conditional Attention":
+//    exact attention over the full context for a sparse subset of queries.
+//  * "Local-global attention", Variants (Gemma 2): causal; the local kind
+//    drops keys more than the window back.
+//
+// One CTA owns two 128-row query tiles that read the same key/value head:
+// two heads of one GQA group on the same rows, or (group size odd) two
+// consecutive row tiles of one head.  Each key/value tile is staged once in
+// shared memory by TMA and feeds both query tiles.
+//
+// Warp roles (10 warps):
+//   warp 0      TMA producer: Q tiles (local mode) and the K/V ring.
+//   warp 1      tcgen05 issuer (one thread): S_i = Q_i K^T into TMEM, then
+//               O_i += P_i V with P_i read straight from TMEM.
+//   warps 2-5   softmax warpgroup for query tile 0 (thread = row = TMEM lane)
+//   warps 6-9   softmax warpgroup for query tile 1
+// TMEM (512 columns): S_0 | S_1 | O_0 | O_1.  P_i (bf16 pairs) overwrites the
+// first half of S_i once the row has been read into registers.
+//
+// Online softmax in fp32 with a lazily updated reference maximum: the
+// accumulator is rescaled only when a row's maximum grows by more than 2^8
+// (in exp2 units), which keeps P <= 256 and exact normalisation at the end.
+//
+// Issue order of the tensor pipe (per key tile j, per query tile i):
+//   PV_i(j), S_i(j+1).  S_i(j+1) overwrites the TMEM columns of P_i(j) only
+//   after PV_i(j) has read them, because tcgen05 MMAs from one thread execute
+//   in issue order; and the commit that signals S_i(j+1) also covers
+//   PV_i(j), so a softmax warpgroup may rescale O_i as soon as it sees S_i(j+1).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cstdint>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace logo {
+
+namespace {
+
+constexpr int kKStages = 2;
+constexpr int kVStages = 2;
+constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
+
+template <int D>
+struct Geometry {
+    static constexpr int kChunks = D / 64;              // 128-byte column chunks of a row
+    static constexpr int kChunkBytes = 128 * 128;       // one chunk of a 128-row tile
+    static constexpr int kQBytes = kTileM * D * 2;
+    static constexpr int kKVBytes = kTileN * D * 2;
+    static constexpr int kQOff = 0;
+    static constexpr int kKOff = kQOff + kNumQ * kQBytes;
+    static constexpr int kVOff = kKOff + kKStages * kKVBytes;
+    static constexpr int kBarOff = kVOff + kVStages * kKVBytes;
+    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 * kNumQ + 2;
+    static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
+    static constexpr int kTmemS = 0;          // S_i at column 128 * i
+    static constexpr int kTmemO = 128 * kNumQ; // O_i at column 256 + D * i
+    static constexpr uint32_t kTmemCols = 512;
+};
+
+// What one CTA computes; identical in every thread.
+struct Work {
+    int valid;
+    int seq;            // sequence index
+    int b;              // batch row of the slab (0 when packed)
+    int s0;             // first row of the sequence in the slab
+    int len;            // sequence length
+    int hk;             // key/value head
+    int head[kNumQ];    // query head of tile i
+    int row0[kNumQ];    // local: first position; global: offset into the selection list
+    int nrows[kNumQ];   // valid rows of tile i
+    int sel_base;       // global: cu_sel[seq]
+    int min_pos, max_pos;
+    int kv_lo, n_kv;
+};
+
+__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+template <int MODE>
+__device__ Work make_work(const AttnParams& p)
+{
+    Work w;
+    w.valid = 0;
+    const int seq = blockIdx.z;
+    w.seq = seq;
+    if (p.cu_seqlens) {
+        w.b = 0;
+        w.s0 = p.cu_seqlens[seq];
+        w.len = p.cu_seqlens[seq + 1] - w.s0;
+    } else {
+        w.b = seq;
+        w.s0 = 0;
+        w.len = p.L;
+    }
+    if (w.len <= 0) return w;
+    if (MODE == kModeLocal) {
+        if (p.pair_heads) {
+            const int tile = gridDim.x - 1 - blockIdx.x;
+            const int t0 = tile * kTileM;
+            if (t0 >= w.len) return w;
+            for (int i = 0; i < kNumQ; ++i) {
+                w.head[i] = blockIdx.y * kNumQ + i;
+                w.row0[i] = t0;
+                w.nrows[i] = min(kTileM, w.len - t0);
+            }
+        } else {
+            const int tile = gridDim.x - 1 - blockIdx.x;
+            const int t0 = tile * kTileM * kNumQ;
+            if (t0 >= w.len) return w;
+            for (int i = 0; i < kNumQ; ++i) {
+                w.head[i] = blockIdx.y;
+                w.row0[i] = t0 + i * kTileM;
+                w.nrows[i] = max(0, min(kTileM, w.len - w.row0[i]));
+            }
+        }
+        w.min_pos = w.row0[0];
+        w.max_pos = w.row0[0];
+        for (int i = 0; i < kNumQ; ++i)
+            if (w.nrows[i] > 0) w.max_pos = max(w.max_pos, w.row0[i] + w.nrows[i] - 1);
+        w.kv_lo = max(0, w.min_pos - p.window + 1);
+    } else {
+        w.sel_base = p.cu_sel[seq];
+        const int k = p.cu_sel[seq + 1] - w.sel_base;
+        if (k > p.max_selected) {
+            if (threadIdx.x == 0) atomicOr(p.status, kStatusBadArgument);
+            return w;
+        }
+        if (k <= 0) return w;
+        const int nch = ceil_div(k, kTileM);
+        if (p.pair_heads) {
+            const int c = nch - 1 - (int)blockIdx.y;
+            if (c < 0) return w;
+            for (int i = 0; i < kNumQ; ++i) {
+                w.head[i] = blockIdx.x * kNumQ + i;
+                w.row0[i] = c * kTileM;
+                w.nrows[i] = min(kTileM, k - c * kTileM);
+            }
+        } else {
+            const int cp = ceil_div(nch, kNumQ) - 1 - (int)blockIdx.y;
+            if (cp < 0) return w;
+            for (int i = 0; i < kNumQ; ++i) {
+                w.head[i] = blockIdx.x;
+                w.row0[i] = (cp * kNumQ + i) * kTileM;
+                w.nrows[i] = max(0, min(kTileM, k - w.row0[i]));
+            }
+        }
+        const int32_t* sel = p.sel_idx + w.sel_base;
+        w.min_pos = sel[w.row0[0]];
+        w.max_pos = w.min_pos;
+        for (int i = 0; i < kNumQ; ++i)
+            if (w.nrows[i] > 0) w.max_pos = max(w.max_pos, sel[w.row0[i] + w.nrows[i] - 1]);
+        w.kv_lo = 0;
+    }
+    w.hk = w.head[0] / p.G;
+    w.n_kv = ceil_div(w.max_pos + 1 - w.kv_lo, kTileN);
+    w.valid = 1;
+    return w;
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p)
+{
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p)
+{
+    using Geo = Geometry<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* sQ = smem + Geo::kQOff;
+    uint8_t* sK = smem + Geo::kKOff;
+    uint8_t* sV = smem + Geo::kVOff;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Geo::kBarOff);
+    uint64_t* q_full = bars;
+    uint64_t* k_full = q_full + 1;
+    uint64_t* k_empty = k_full + kKStages;
+    uint64_t* v_full = k_empty + kKStages;
+    uint64_t* v_empty = v_full + kVStages;
+    uint64_t* s_full = v_empty + kVStages;
+    uint64_t* p_full = s_full + kNumQ;
+    uint64_t* o_full = p_full + kNumQ;
+    uint64_t* drain = o_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // A CTA launched after another one recorded a timeout does no work, so a
+    // broken launch ends quickly instead of waiting out every CTA's limit.
+    __shared__ int sh_skip;
+    if (threadIdx.x == 0) sh_skip = (*reinterpret_cast<volatile uint32_t*>(p.status) & kStatusTimeout) ? 1 : 0;
+    __syncthreads();
+    if (sh_skip) return;
+
+    const Work w = make_work<MODE>(p);
+    if (!w.valid) return;  // uniform across the CTA
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, MODE == kModeLocal ? 1 : 128 * kNumQ);
+        for (int s = 0; s < kKStages; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
+        }
+        for (int i = 0; i < kNumQ; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], 128);
+        }
+        mbar_init(o_full, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, Geo::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint64_t limit = p.timeout_ns;
+    const int n_kv = w.n_kv;
+    const int zkv = w.b * p.Hkv + w.hk;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&p.tm_k);
+            tma_prefetch_desc(&p.tm_v);
+            const uint64_t pol_kv = policy_evict_last();
+            bool ok = true;
+            if (MODE == kModeLocal) {
+                tma_prefetch_desc(&p.tm_q);
+                const uint64_t pol_q = policy_evict_first();
+                mbar_arrive_expect_tx(q_full, kNumQ * Geo::kQBytes);
+                for (int i = 0; i < kNumQ; ++i)
+                    for (int c = 0; c < Geo::kChunks; ++c)
+                        tma_load_3d(sQ + i * Geo::kQBytes + c * Geo::kChunkBytes, &p.tm_q, q_full, c * 64,
+                                    w.s0 + w.row0[i], w.b * p.Hq + w.head[i], pol_q);
+            }
+            int k_armed[kKStages], v_armed[kVStages];
+            for (int s = 0; s < kKStages; ++s) k_armed[s] = 0;
+            for (int s = 0; s < kVStages; ++s) v_armed[s] = 0;
+            for (int j = 0; j < n_kv && ok; ++j) {
+                const int row = w.s0 + w.kv_lo + j * kTileN;
+                const int ks = j % kKStages;
+                if (j >= kKStages) ok = mbar_wait(&k_empty[ks], ((j / kKStages) - 1) & 1, abort_flag, p.status, limit);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&k_full[ks], Geo::kKVBytes);
+                ++k_armed[ks];
+                for (int c = 0; c < Geo::kChunks; ++c)
+                    tma_load_3d(sK + ks * Geo::kKVBytes + c * Geo::kChunkBytes, &p.tm_k, &k_full[ks], c * 64, row,
+                                zkv, pol_kv);
+                const int vs = j % kVStages;
+                if (j >= kVStages) ok = mbar_wait(&v_empty[vs], ((j / kVStages) - 1) & 1, abort_flag, p.status, limit);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&v_full[vs], Geo::kKVBytes);
+                ++v_armed[vs];
+                for (int c = 0; c < Geo::kChunks; ++c)
+                    tma_load_3d(sV + vs * Geo::kKVBytes + c * Geo::kChunkBytes, &p.tm_v, &v_full[vs], c * 64, row,
+                                zkv, pol_kv);
+            }
+            if (*abort_flag) {
+                // Let every copy this thread started land before the CTA exits.
+                volatile int dummy = 0;
+                for (int s = 0; s < kKStages; ++s)
+                    if (k_armed[s]) mbar_wait(&k_full[s], (k_armed[s] - 1) & 1, &dummy, nullptr, limit);
+                for (int s = 0; s < kVStages; ++s)
+                    if (v_armed[s]) mbar_wait(&v_full[s], (v_armed[s] - 1) & 1, &dummy, nullptr, limit);
+                if (MODE == kModeLocal) mbar_wait(q_full, 0, &dummy, nullptr, limit);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ tcgen05 issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(kTileM, kTileN, false);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(kTileM, D, true);
+            const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+            auto issue_s = [&](int i, int ks) {
+                const uint32_t d_tmem = tmem + Geo::kTmemS + 128 * i;
+                #pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * Geo::kChunkBytes + (kk & 3) * 32;
+                    const uint64_t a = sdesc_sw128(sQa + i * Geo::kQBytes + off, 16, 1024);
+                    const uint64_t b = sdesc_sw128(sKa + ks * Geo::kKVBytes + off, 16, 1024);
+                    umma_ss(d_tmem, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_pv = [&](int i, int vs, bool first) {
+                const uint32_t d_tmem = tmem + Geo::kTmemO + D * i;
+                const uint32_t p_tmem = tmem + Geo::kTmemS + 128 * i;
+                #pragma unroll
+                for (int kk = 0; kk < kTileN / 16; ++kk) {
+                    const uint64_t b = sdesc_sw128(sVa + vs * Geo::kKVBytes + kk * 2048, Geo::kChunkBytes, 1024);
+                    umma_ts(d_tmem, p_tmem + kk * 8, b, idesc_pv, (!first || kk > 0) ? 1u : 0u);
+                }
+            };
+            bool ok = mbar_wait(q_full, 0, abort_flag, p.status, limit);
+            if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag, p.status, limit);
+            if (ok) {
+                tc_fence_after();
+                for (int i = 0; i < kNumQ; ++i) {
+                    issue_s(i, 0);
+                    umma_commit(&s_full[i]);
+                }
+                umma_commit(&k_empty[0]);
+            }
+            for (int j = 0; j < n_kv && ok; ++j) {
+                const bool nxt = j + 1 < n_kv;
+                const int ks1 = (j + 1) % kKStages;
+                const int vs = j % kVStages;
+                if (nxt) ok = mbar_wait(&k_full[ks1], ((j + 1) / kKStages) & 1, abort_flag, p.status, limit);
+                if (ok) ok = mbar_wait(&v_full[vs], (j / kVStages) & 1, abort_flag, p.status, limit);
+                if (!ok) break;
+                tc_fence_after();
+                for (int i = 0; i < kNumQ && ok; ++i) {
+                    ok = mbar_wait(&p_full[i], j & 1, abort_flag, p.status, limit);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(i, vs, j == 0);
+                    if (nxt) {
+                        issue_s(i, ks1);
+                        umma_commit(&s_full[i]);
+                    }
+                }
+                if (!ok) break;
+                if (nxt) umma_commit(&k_empty[ks1]);
+                umma_commit(&v_empty[vs]);
+            }
+            if (ok) umma_commit(o_full);
+            // Drain: everything issued above completes before TMEM is released.
+            umma_commit(drain);
+            volatile int dummy = 0;
+            mbar_wait(drain, 0, &dummy, nullptr, limit);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax warpgroups
+        const int wg = (warp - 2) >> 2;          // query tile
+        const int quarter = warp & 3;             // TMEM lane quarter this warp may touch
+        const int r = quarter * 32 + lane;        // row of the tile = TMEM lane
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const uint32_t tS = tmem + lane_off + Geo::kTmemS + 128 * wg;
+        const uint32_t tO = tmem + lane_off + Geo::kTmemO + D * wg;
+        const bool row_valid = r < w.nrows[wg];
+        const int head = w.head[wg];
+        const int zq = w.b * p.Hq + head;
+        int pos;  // position of this row within its sequence
+        if (MODE == kModeLocal) {
+            pos = row_valid ? w.row0[wg] + r : w.max_pos;
+        } else {
+            pos = row_valid ? p.sel_idx[w.sel_base + w.row0[wg] + r] : w.max_pos;
+            // Gather this row of Q into the 128B-swizzled tile.
+            uint8_t* dst = sQ + wg * Geo::kQBytes;
+            const int4* src = reinterpret_cast<const int4*>(p.q + ((size_t)zq * p.L + w.s0 + pos) * D);
+            #pragma unroll
+            for (int c = 0; c < Geo::kChunks; ++c) {
+                #pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    int4 val = row_valid ? __ldg(src + c * 8 + u) : make_int4(0, 0, 0, 0);
+                    *reinterpret_cast<int4*>(dst + c * Geo::kChunkBytes + r * 128 + ((u ^ (r & 7)) << 4)) = val;
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(q_full);
+        }
+        const float sl2 = p.scale_log2;
+        const float resc_raw = kRescaleLog2 / sl2;  // threshold in raw score units
+        float m_run = -INFINITY;  // reference max (raw units)
+        float l_run = 0.f;
+        bool ok = true;
+        const int W = p.window;
+        for (int j = 0; j < n_kv; ++j) {
+            // Warp-uniform outcome: the tcgen05 loads below are warp-collective.
+            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], j & 1, abort_flag, p.status, limit));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t sr[4][32];
+            #pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+            #pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_wait_ld(sr[c]);
+            const int kbase = w.kv_lo + j * kTileN;
+            const bool need_mask = (kbase + kTileN - 1 > w.min_pos) ||
+                                   (MODE == kModeLocal && kbase < w.max_pos - W + 1);
+            if (need_mask) {
+                const int hi = pos - kbase;                                       // keep c <= hi
+                const int lo = (MODE == kModeLocal) ? pos - W + 1 - kbase : INT_MIN; // keep c >= lo
+                #pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    #pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int col = c * 32 + e;
+                        if (col > hi || col < lo) sr[c][e] = __float_as_uint(-INFINITY);
+                    }
+                }
+            }
+            float mt = -INFINITY;
+            #pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                #pragma unroll
+                for (int e = 0; e < 32; ++e) mt = fmaxf(mt, __uint_as_float(sr[c][e]));
+            }
+            const float m_new = fmaxf(m_run, mt);
+            const bool need = m_new > m_run + resc_raw;
+            float alpha = 1.f;
+            if (need) {
+                alpha = (m_run == -INFINITY) ? 0.f : fast_exp2((m_run - m_new) * sl2);
+                m_run = m_new;
+                l_run *= alpha;
+            }
+            const bool any = __any_sync(0xffffffffu, need);  // also reconverges the warp
+            if (any && j > 0) {
+                // Rescale this warp's rows of O (PV of tile j-1 is complete: see header).
+                #pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t orr[32];
+                    tmem_ld32(tO + c * 32, orr);
+                    tmem_wait_ld(orr);
+                    #pragma unroll
+                    for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                    tmem_st32(tO + c * 32, orr);
+                }
+            }
+            const float mref = (m_run == -INFINITY) ? 0.f : m_run * sl2;
+            uint32_t pk[64];
+            float lsum = 0.f;
+            #pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                #pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c][e]), sl2, -mref));
+                    const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c][e + 1]), sl2, -mref));
+                    lsum += p0 + p1;
+                    pk[c * 16 + e / 2] = pack_bf16x2(p0, p1);
+                }
+            }
+            l_run += lsum;
+            __syncwarp();
+            tmem_st32(tS, pk);
+            tmem_st32(tS + 32, pk + 32);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&p_full[wg]);
+        }
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, abort_flag, p.status, limit));
+        if (ok) {
+            tc_fence_after();
+            const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+            uint16_t* orow = p.out + ((size_t)zq * p.L + w.s0 + pos) * D;
+            float gsig = 0.f;
+            if (MODE == kModeGlobal && p.merge && row_valid) {
+                const float g = p.gate[(size_t)w.b * p.L + w.s0 + pos];
+                gsig = 1.f / (1.f + expf(-g));
+            }
+            #pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t orr[32];
+                __syncwarp();
+                tmem_ld32(tO + c * 32, orr);
+                tmem_wait_ld(orr);
+                if (!row_valid) continue;
+                float vals[32];
+                #pragma unroll
+                for (int e = 0; e < 32; ++e) vals[e] = __uint_as_float(orr[e]) * inv_l;
+                int4* dst = reinterpret_cast<int4*>(orow + c * 32);
+                if (MODE == kModeGlobal && p.merge) {
+                    #pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        int4 loc = dst[u];
+                        const uint32_t lw[4] = {(uint32_t)loc.x, (uint32_t)loc.y, (uint32_t)loc.z, (uint32_t)loc.w};
+                        #pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            const float lo = __uint_as_float(lw[t] << 16);
+                            const float hi = __uint_as_float(lw[t] & 0xffff0000u);
+                            vals[u * 8 + 2 * t] = fmaf(gsig, vals[u * 8 + 2 * t], lo);
+                            vals[u * 8 + 2 * t + 1] = fmaf(gsig, vals[u * 8 + 2 * t + 1], hi);
+                        }
+                    }
+                }
+                #pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    int4 o;
+                    o.x = (int)pack_bf16x2(vals[u * 8 + 0], vals[u * 8 + 1]);
+                    o.y = (int)pack_bf16x2(vals[u * 8 + 2], vals[u * 8 + 3]);
+                    o.z = (int)pack_bf16x2(vals[u * 8 + 4], vals[u * 8 + 5]);
+                    o.w = (int)pack_bf16x2(vals[u * 8 + 6], vals[u * 8 + 7]);
+                    dst[u] = o;
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, Geo::kTmemCols);
+    }
+}
+
+template <int D, int MODE>
+cudaError_t launch_one(const AttnParams& p, dim3 grid, cudaStream_t stream)
+{
+    const size_t smem = Geometry<D>::kBytes + 1024;
+    auto kern = attn_fwd_kernel<D, MODE>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t attn_smem_bytes(int d)
+{
+    return d == 64 ? Geometry<64>::kBytes + 1024 : Geometry<128>::kBytes + 1024;
+}
+
+cudaError_t launch_attn(int mode, int d, const AttnParams& p, int max_seqlen, cudaStream_t stream)
+{
+    dim3 grid;
+    if (mode == kModeLocal) {
+        const int tiles = p.pair_heads ? (max_seqlen + kTileM - 1) / kTileM
+                                       : (max_seqlen + kTileM * kNumQ - 1) / (kTileM * kNumQ);
+        grid = dim3(tiles, p.pair_heads ? p.Hq / kNumQ : p.Hq, p.nseq);
+    } else {
+        const int nch = (p.max_selected + kTileM - 1) / kTileM;
+        grid = p.pair_heads ? dim3(p.Hq / kNumQ, nch, p.nseq)
+                            : dim3(p.Hq, (nch + kNumQ - 1) / kNumQ, p.nseq);
+    }
+    if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
+    if (d == 64)
+        return mode == kModeLocal ? launch_one<64, kModeLocal>(p, grid, stream)
+                                  : launch_one<64, kModeGlobal>(p, grid, stream);
+    return mode == kModeLocal ? launch_one<128, kModeLocal>(p, grid, stream)
+                              : launch_one<128, kModeGlobal>(p, grid, stream);
+}
+
+// ---------------------------------------------------------------- timeout probe
+
+__global__ void timeout_probe_kernel(uint32_t* status, unsigned long long limit_ns)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);  // nothing ever arrives
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, status, limit_ns);
+}
+
+cudaError_t launch_timeout_probe(uint32_t* status, unsigned long long limit_ns, cudaStream_t stream)
+{
+    timeout_probe_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace logo

@@ -1,0 +1,76 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace logo {
+
+// Device-side status word bits (first word of the caller's workspace).
+enum : uint32_t {
+    kStatusTimeout = 1u,      // a bounded wait ran out
+    kStatusBadArgument = 2u,  // a kernel met an argument it cannot handle
+};
+
+// Budget count, identical on host and device (see logo_num_selected in
+// logo.h).  The product is formed with an explicit round-to-nearest multiply
+// so device code cannot contract it into a fused multiply-add.
+__host__ __device__ inline int64_t budget_count(double ratio, int64_t len)
+{
+    if (len <= 0 || !(ratio > 0.0)) return 0;
+#ifdef __CUDA_ARCH__
+    const double x = __dmul_rn(ratio, (double)len);
+    const double r = rint(x);
+    const double diff = fabs(__dadd_rn(x, -r));
+#else
+    volatile double xv = ratio * (double)len;  // no contraction on the host either
+    const double x = xv;
+    const double r = nearbyint(x);
+    const double diff = fabs(x - r);
+#endif
+    const double tol = 1e-9 * (x > 1.0 ? x : 1.0);
+    double kk = (diff <= tol) ? r : ceil(x);
+    if (kk < 0.0) kk = 0.0;
+    if (kk > (double)len) kk = (double)len;
+    return (int64_t)kk;
+}
+
+constexpr int kTileM = 128;   // query rows per Q tile (= TMEM lanes)
+constexpr int kTileN = 128;   // keys per K/V tile
+constexpr int kNumQ = 2;      // Q tiles per CTA, one softmax warpgroup each
+constexpr int kThreads = 64 + 128 * kNumQ;
+
+enum AttnMode : int { kModeLocal = 0, kModeGlobal = 1 };
+
+struct alignas(64) AttnParams {
+    CUtensorMap tm_q;   // Q as [B*Hq][L][d] (local mode loads Q tiles by TMA)
+    CUtensorMap tm_k;   // K as [B*Hkv][L][d]
+    CUtensorMap tm_v;   // V as [B*Hkv][L][d]
+    const uint16_t* q;  // raw Q (global mode gathers selected rows)
+    uint16_t* out;
+    const float* gate;
+    const int32_t* cu_seqlens;  // nullptr: fixed length
+    const int32_t* sel_idx;
+    const int32_t* cu_sel;
+    uint32_t* status;
+    int Hq, Hkv, G;
+    int L;          // rows per head slab (L, or T when packed)
+    int nseq;
+    int window;
+    int pair_heads; // 1: the CTA's Q tiles are heads (h, h+1) on the same rows
+    int max_selected;
+    int merge;
+    float scale_log2;  // softmax scale * log2(e)
+    unsigned long long timeout_ns;
+};
+
+cudaError_t launch_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, double ratio,
+                          int32_t* sel_idx, int32_t* cu_sel, cudaStream_t stream);
+
+cudaError_t launch_attn(int mode, int d, const AttnParams& p, int max_seqlen, cudaStream_t stream);
+
+cudaError_t launch_timeout_probe(uint32_t* status, unsigned long long limit_ns, cudaStream_t stream);
+
+size_t attn_smem_bytes(int d);
+
+}  // namespace logo

@@ -1,0 +1,208 @@
+// Budget rule on the GPU: per sequence, the k = budget_count(ratio, len)
+// positions with the largest gate logits, ties to the lower position, emitted
+// in ascending order.
+//
+// Sources: "LoGo: Token-Level Dynamic Local-Global Attention", Abstract (a
+// learned gate activates global attention for some tokens; a budget
+// controller keeps a target global ratio); "Learning When to Attend", "The
+// Architecture of Conditional Attention" (one binary decision per token,
+// about 20% of tokens global).
+//
+// One 1024-thread CTA per sequence:
+//  1. map each fp32 logit to a 32-bit key whose unsigned order is the
+//     selection order (-0 folded onto +0, every NaN to 0, below -inf);
+//  2. radix-select the k-th largest key T with four 8-bit passes
+//     (warp-aggregated shared-memory histograms), which also yields how many
+//     keys equal to T must be taken;
+//  3. stream-compact in ascending position order with two block-wide scans
+//     per 4096-element chunk: one ranks the keys equal to T (the lowest
+//     positions win), the other places the selected positions.
+// Integer work only, so the result is bit-exact.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kernels.cuh"
+
+namespace logo {
+
+namespace {
+
+constexpr int kSelThreads = 1024;
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kItems = 4;
+
+__device__ __forceinline__ uint32_t gate_key(float f)
+{
+    uint32_t b = __float_as_uint(f);
+    if ((b & 0x7FFFFFFFu) > 0x7F800000u) return 0u;  // NaN ranks below everything
+    if (b == 0x80000000u) b = 0u;                      // -0 equals +0
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Exclusive prefix sum over the block; `total` receives the block sum.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_buf, int& total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+    #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_buf[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int s = warp_buf[lane];
+        #pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += y;
+        }
+        warp_buf[lane] = s;  // inclusive
+    }
+    __syncthreads();
+    const int before = warp ? warp_buf[warp - 1] : 0;
+    total = warp_buf[kSelWarps - 1];
+    __syncthreads();  // warp_buf may be reused right after
+    return before + x - v;
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const float* __restrict__ gate,
+                                                                  const int32_t* __restrict__ cu_seqlens,
+                                                                  int nseq, int L, double ratio,
+                                                                  int32_t* __restrict__ sel_idx,
+                                                                  int32_t* __restrict__ cu_sel)
+{
+    __shared__ uint32_t hist[256];
+    __shared__ int warp_buf[32];
+    __shared__ uint32_t sh_digit;
+    __shared__ long long sh_remaining;
+
+    const int s = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    long long start, len, out_off;
+    if (cu_seqlens) {
+        start = cu_seqlens[s];
+        len = (long long)cu_seqlens[s + 1] - start;
+        out_off = 0;
+        for (int t = 0; t < s; ++t) out_off += budget_count(ratio, (long long)cu_seqlens[t + 1] - cu_seqlens[t]);
+    } else {
+        start = (long long)s * L;
+        len = L;
+        out_off = (long long)s * budget_count(ratio, L);
+    }
+    const long long k = budget_count(ratio, len);
+    if (tid == 0) {
+        cu_sel[s + 1] = (int32_t)(out_off + k);
+        if (s == 0) cu_sel[0] = 0;
+    }
+    if (k <= 0) return;
+    const float* g = gate + start;
+    int32_t* out = sel_idx + out_off;
+    if (k == len) {
+        for (long long i = tid; i < len; i += kSelThreads) out[i] = (int32_t)i;
+        return;
+    }
+
+    // ---- radix select of the k-th largest key
+    uint32_t prefix = 0, mask = 0;
+    long long remaining = k;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
+        __syncthreads();
+        for (long long base = (long long)warp * 32; base < len; base += kSelThreads) {
+            const long long i = base + lane;
+            const bool in = i < len;
+            const uint32_t key = in ? gate_key(g[i]) : 0u;
+            const bool match = in && ((key & mask) == prefix);
+            const uint32_t digit = (key >> shift) & 255u;
+            const uint32_t tag = match ? digit : 256u + lane;  // unmatched lanes stay alone
+            const uint32_t peers = __match_any_sync(0xffffffffu, tag);
+            if (match && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (uint32_t)__popc(peers));
+        }
+        __syncthreads();
+        if (warp == 0) {
+            // lane l owns bins 255-8l .. 248-8l (descending)
+            uint32_t c[8];
+            uint32_t sum = 0;
+            #pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                c[t] = hist[255 - 8 * lane - t];
+                sum += c[t];
+            }
+            uint32_t incl = sum;
+            #pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const long long excl = (long long)(incl - sum);
+            if (excl < remaining && remaining <= excl + (long long)sum) {
+                long long acc = excl;
+                #pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    if (acc + (long long)c[t] >= remaining) {
+                        sh_digit = 255u - 8u * lane - t;
+                        sh_remaining = remaining - acc;
+                        break;
+                    }
+                    acc += c[t];
+                }
+            }
+        }
+        __syncthreads();
+        prefix |= sh_digit << shift;
+        mask |= 255u << shift;
+        remaining = sh_remaining;
+        __syncthreads();
+    }
+    const uint32_t T = prefix;           // the k-th largest key
+    const long long take_eq = remaining; // how many keys equal to T are selected
+
+    // ---- compaction in ascending position order
+    long long eq_seen = 0, written = 0;
+    for (long long chunk = 0; chunk < len; chunk += (long long)kSelThreads * kItems) {
+        const long long i0 = chunk + (long long)tid * kItems;
+        uint32_t keys[kItems];
+        int n_eq = 0;
+        #pragma unroll
+        for (int t = 0; t < kItems; ++t) {
+            keys[t] = (i0 + t < len) ? gate_key(g[i0 + t]) : 0u;
+            n_eq += (i0 + t < len && keys[t] == T) ? 1 : 0;
+        }
+        int eq_total;
+        const int eq_before = block_exclusive_scan(n_eq, warp_buf, eq_total);
+        bool sel[kItems];
+        int n_sel = 0, eq_run = 0;
+        #pragma unroll
+        for (int t = 0; t < kItems; ++t) {
+            const bool in = i0 + t < len;
+            const bool gt = in && keys[t] > T;
+            const bool eq = in && keys[t] == T;
+            sel[t] = gt || (eq && (eq_seen + eq_before + eq_run) < take_eq);
+            eq_run += eq ? 1 : 0;
+            n_sel += sel[t] ? 1 : 0;
+        }
+        int sel_total;
+        const int sel_before = block_exclusive_scan(n_sel, warp_buf, sel_total);
+        int o = 0;
+        #pragma unroll
+        for (int t = 0; t < kItems; ++t)
+            if (sel[t]) out[written + sel_before + (o++)] = (int32_t)(i0 + t);
+        eq_seen += eq_total;
+        written += sel_total;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, double ratio,
+                          int32_t* sel_idx, int32_t* cu_sel, cudaStream_t stream)
+{
+    if (nseq <= 0) return cudaSuccess;
+    select_topk_kernel<<<nseq, kSelThreads, 0, stream>>>(gate, cu_seqlens, nseq, L, ratio, sel_idx, cu_sel);
+    return cudaGetLastError();
+}
+
+}  // namespace logo
