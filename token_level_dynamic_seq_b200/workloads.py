@@ -112,6 +112,9 @@ CONFIGS = {
     "c4k": dict(B=2, Hq=8, Hkv=8, L=4096, d=128, W=512, ratio=0.2, qkv_scale=128 ** -0.5),
     "c32k": dict(B=1, Hq=32, Hkv=8, L=32768, d=128, W=4096, ratio=0.2, qkv_scale=1.0),
 }
+# The headline shape at a quarter of the length: inputs still larger than L2,
+# small enough for a many-pass profiler capture.
+CONFIGS["c8k"] = dict(B=1, Hq=32, Hkv=8, L=8192, d=128, W=4096, ratio=0.2, qkv_scale=1.0)
 for _r in RATIO_SWEEP_128K:
     CONFIGS[f"c128k_r{_r:g}"] = dict(B=1, Hq=32, Hkv=8, L=131072, d=128, W=4096, ratio=_r,
                                      qkv_scale=1.0)
@@ -137,14 +140,12 @@ def describe(name: str) -> str:
 
 
 def load(name: str, seed: int = 0) -> Workload:
-    """Build a named workload: tiny, c4k, c32k (headline), c128k_r{ratio}, varlen."""
+    """Build a named workload: tiny, c4k, c8k, c32k (headline), c128k_r{ratio}, varlen."""
     if name == "varlen":
-        # One generator for the whole workload: lengths, then Q, K, V, g, bursts.
-        gen_seed = seed
-        lens = varlen_seqlens(gen_seed)
-        # The lengths consumed the first draws of the seed; Q/K/V/g use seed + 1 so the
-        # two streams stay independent of each other's sizes.
-        w = make(1, 32, 8, 0, 128, 2048, 0.25, seed=gen_seed + 1, qkv_scale=1.0, seqlens=lens,
+        # Lengths come from a generator seeded with `seed`; Q, K, V, the gate
+        # logits and the burst starts (in that order) from one seeded with seed + 1.
+        lens = varlen_seqlens(seed)
+        w = make(1, 32, 8, 0, 128, 2048, 0.25, seed=seed + 1, qkv_scale=1.0, seqlens=lens,
                  burst_p=0.01, burst_len=64, burst_add=3.0, name="varlen")
     else:
         c = dict(CONFIGS[name])
