@@ -2,7 +2,7 @@
 
 Workload (N = 1): B=1, Hq=32, Hkv=8 (GQA), L=32768, d=128, W=4096, ratio 0.2,
 bf16 N(0,1) Q/K/V, fp32 N(0,1) gate logits (seeded, synthetic).  One step is
-one pass of the whole hot path: selection, local attention, query-sparse
+one pass of the whole hot path: selection, local attention, selected-query
 global attention with the fused gated merge, launched through the C ABI on one
 stream.  With --gpus N (torchrun), every rank runs its own independent
 sequence (seed = rank): weak scaling, no collective on the data path; the

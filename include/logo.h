@@ -3,19 +3,19 @@
  * pass of token-level dynamic local-global attention (LoGo / L2A).
  *
  * What the library computes, and where the pages define it:
- *   - "LoGo: Token-Level Dynamic Local-Global Attention", Abstract: each layer
- *     has a local and a global branch; every token gets local attention over
- *     a restricted window; a learned gate gives full-context attention only
- *     to the tokens that need it; a budget controller keeps a target global
- *     ratio; query-sparse kernels turn the reduced global work into speed.
+ *   - "LoGo: Token-Level Dynamic Local-Global Attention", Abstract: a layer
+ *     couples a windowed branch, computed for every token, with a
+ *     whole-prefix branch that a gate switches on token by token; the share
+ *     of switched-on tokens is held at a set value; the kernels skip the
+ *     global work of the other queries.
  *   - "Learning When to Attend", "The Architecture of Conditional Attention":
- *     local attention over a fixed recent window for all tokens, then exact
- *     attention over the full context for a sparse subset of query tokens
- *     (about 20% of them).
+ *     windowed attention for all positions, and exact softmax attention over
+ *     everything before a position only at the routed positions (about one
+ *     in five).
  *   - "Local-global attention", Variants, Gemma 2: attention is causal and the
- *     local kind drops keys more than the window back; Implementation sketch
- *     notes, "Packed examples (LongT5)": packed examples must be masked per
- *     example.
+ *     windowed kind ignores keys further back than the window; Implementation
+ *     sketch notes, "Packed examples (LongT5)": sequences packed together
+ *     must not see each other.
  * Readings of what the pages leave open (fixed here, identical in every entry
  * point):
  *   - window: query i attends to key j iff 0 <= i - j < W;
@@ -98,7 +98,8 @@ typedef struct {
 } logo_shape;
 
 /*
- * Budget count for one sequence ("LoGo", Abstract: target global ratio):
+ * Budget count for one sequence ("LoGo", Abstract: the share of tokens on the
+ * global branch is held at a set value):
  * k = ceil(ratio * len), computed in double; a product within 1e-9
  * (relative, absolute at least 1e-9) of an integer is taken as that integer,
  * so 0.07 * 100 gives 7, not 8.  Clamped to [0, len].  Host function; never
@@ -135,10 +136,10 @@ LOGO_API logo_status logo_select(const float *gate, const logo_shape *shape, dou
                         int32_t *cu_sel, void *ws, size_t ws_bytes, logo_stream_t stream);
 
 /*
- * Local branch for every query ("LoGo", Abstract: local attention over a
- * restricted window; "Learning When to Attend": a fixed recent window;
- * "Local-global attention", Gemma 2 variant: causal, keys more than W back
- * dropped): out[b, h, i] = softmax_j(scale * q_i . k_j) v_j over keys j of
+ * Local branch for every query ("LoGo", Abstract: the windowed branch runs
+ * for every token; "Learning When to Attend": each position looks back over
+ * a window of fixed size; "Local-global attention", Gemma 2 variant: causal,
+ * keys further back than the window ignored): out[b, h, i] = softmax_j(scale * q_i . k_j) v_j over keys j of
  * the same sequence with 0 <= i - j < W.  With W >= L this is dense causal
  * attention.  q, k, v, out as in logo_shape; `scale` <= 0 means 1/sqrt(d).
  */
@@ -147,10 +148,11 @@ LOGO_API logo_status logo_local_attn(const logo_bf16 *q, const logo_bf16 *k, con
                             size_t ws_bytes, logo_stream_t stream);
 
 /*
- * Query-sparse global branch and gated merge ("Learning When to Attend", "The
- * Architecture of Conditional Attention": exact attention over the full
- * context for a sparse subset of query tokens; "LoGo", Abstract: query-sparse
- * kernels).  For every selected position i of sequence s (from sel_idx /
+ * Global branch on the selected queries only, and the gated merge ("Learning
+ * When to Attend", "The Architecture of Conditional Attention": exact softmax
+ * attention over everything before a position, run only at the routed
+ * positions; "LoGo", Abstract: kernels that skip the global work of the other
+ * queries).  For every selected position i of sequence s (from sel_idx /
  * cu_sel, as written by logo_select) and every query head h:
  *   global = softmax_j(scale * q_i . k_j) v_j over keys 0..i of sequence s;
  *   merge != 0: out[i] = out[i] + sigmoid(gate[i]) * global  (out must hold

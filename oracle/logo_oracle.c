@@ -9,17 +9,16 @@
  * helper with the CUDA library.
  *
  * What it computes (sources are the pages' titles and sections):
- *   - "LoGo: Token-Level Dynamic Local-Global Attention", Abstract: every
- *     token gets local attention over a restricted window; a learned gate
- *     turns on full-context (global) attention for a subset of tokens; a
- *     budget controller keeps a target global ratio.
+ *   - "LoGo: Token-Level Dynamic Local-Global Attention", Abstract: each
+ *     layer pairs a windowed branch, run for every token, with a whole-prefix
+ *     branch that a gate switches on per token; the share of switched-on
+ *     tokens is held at a set fraction.
  *   - "Learning When to Attend", section "The Architecture of Conditional
- *     Attention": local attention over a fixed recent window for all tokens,
- *     then exact attention over the full context for a sparse subset of query
- *     tokens only.
+ *     Attention": the windowed pass runs for all positions; the unrestricted
+ *     pass is exact softmax attention, run only at the chosen positions.
  *   - "Local-global attention", Variants, "Alternating sliding-window and
- *     global layers (Gemma 2)": both kinds are causal; the local kind drops
- *     keys more than the window back.
+ *     global layers (Gemma 2)": both kinds are causal; the windowed kind
+ *     ignores keys that lie further back than the window.
  *   - "Local-global attention", Implementation sketch, notes, "Packed examples
  *     (LongT5)": packed examples must not attend to one another.
  *
@@ -65,12 +64,13 @@ static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
 
 /*
  * Budget: the number of query tokens that take the global branch in a
- * sequence of `len` tokens at target ratio `ratio` ("LoGo", Abstract: a
- * budget controller keeps a target global ratio; "Learning When to Attend",
- * "The Architecture of Conditional Attention": about 20% of tokens).
+ * sequence of `len` tokens at ratio `ratio` ("LoGo", Abstract: the share of
+ * tokens on the global branch is held at a set value; "Learning When to
+ * Attend", "The Architecture of Conditional Attention": about one token in
+ * five).
  * Reading: k = ceil(ratio * len).  The product is formed in double; when it
  * lies within 1e-9 (relative, at least absolute 1e-9) of an integer it is
- * taken as that integer, so that 0.2 * 5 = 1.0000000000000002 gives 1, not 2.
+ * taken as that integer, so that 0.07 * 100 = 7.000000000000001 gives 7, not 8.
  * The result is clamped to [0, len].
  */
 int64_t oracle_num_selected(double ratio, int64_t len)

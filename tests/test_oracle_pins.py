@@ -13,8 +13,9 @@ The oracle is trusted only because it agrees with things other than itself:
 Sources of the method (page titles and sections):
   "LoGo: Token-Level Dynamic Local-Global Attention", Abstract;
   "Learning When to Attend", "The Architecture of Conditional Attention";
-  "Local-global attention", Variants (Gemma 2: causal, keys more than the
-  window back dropped) and Implementation sketch notes (packed examples).
+  "Local-global attention", Variants (Gemma 2: causal; the windowed kind
+  ignores keys further back than the window) and Implementation sketch notes
+  (packed examples).
 """
 import math
 import os

@@ -1,15 +1,16 @@
-// Local (sliding-window) and query-sparse global attention forward kernels
-// for sm_100a, with the gated merge fused into the global kernel's epilogue.
+// Local (sliding-window) and selected-query global attention forward
+// kernels for sm_100a, with the gated merge fused into the global kernel's
+// epilogue.
 //
 // Method sources (page titles and sections):
-//  * "LoGo: Token-Level Dynamic Local-Global Attention", Abstract: all tokens
-//    get local attention over a restricted window; a gate activates
-//    full-context attention only for some tokens; query-sparse kernels turn
-//    the reduced global work into speed.
+//  * "LoGo: Token-Level Dynamic Local-Global Attention", Abstract: a windowed
+//    branch for every token, a whole-prefix branch only where a gate turns it
+//    on, and kernels that skip the global work of the other queries.
 //  * "Learning When to Attend", "The Architecture of Conditional Attention":
-//    exact attention over the full context for a sparse subset of queries.
-//  * "Local-global attention", Variants (Gemma 2): causal; the local kind
-//    drops keys more than the window back.
+//    the global branch is exact softmax attention, evaluated only at the
+//    chosen query positions.
+//  * "Local-global attention", Variants (Gemma 2): causal; the windowed kind
+//    ignores keys further back than the window.
 //
 // One CTA owns two 128-row query tiles that read the same key/value head:
 // two heads of one GQA group on the same rows, or (group size odd) two

@@ -3,10 +3,10 @@
 // in ascending order.
 //
 // Sources: "LoGo: Token-Level Dynamic Local-Global Attention", Abstract (a
-// learned gate activates global attention for some tokens; a budget
-// controller keeps a target global ratio); "Learning When to Attend", "The
-// Architecture of Conditional Attention" (one binary decision per token,
-// about 20% of tokens global).
+// gate decides per token whether the global branch runs; the share of such
+// tokens is held at a set value); "Learning When to Attend", "The
+// Architecture of Conditional Attention" (a yes/no routing decision for each
+// position, about one in five going global).
 //
 // One 1024-thread CTA per sequence:
 //  1. map each fp32 logit to a 32-bit key whose unsigned order is the
