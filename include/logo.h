@@ -181,6 +181,29 @@ LOGO_API logo_status logo_forward(const logo_bf16 *q, const logo_bf16 *k, const 
                          logo_stream_t stream);
 
 /*
+ * The same computation as logo_global_attn_sparse (same arguments, same
+ * results) for callers that cannot allocate device memory: a layer that only
+ * receives the op's tensors from a framework whose allocator owns the device
+ * (and cannot ask it for a workspace), or a serving loop where cudaMalloc /
+ * cudaFree would synchronise the device.  No counterpart in the pages: it is
+ * a property of this library's interface.
+ * Scratch: instead of a caller workspace, a fixed 256 KiB array compiled into
+ * the library, held on every GPU that loads the library until exit.  Shapes
+ * whose workspace (logo_workspace_size at ratio 1) exceeds it are refused with
+ * LOGO_ERR_WORKSPACE.  The first call on a device looks the array's address up
+ * (once per device, with that device current): make it before any stream
+ * capture.  All calls on a device share the array; each call clears its
+ * status word first, and calls that overlap on the GPU race on it.  Device
+ * errors of a call are recorded there but cannot be read back: use
+ * logo_global_attn_sparse and logo_check when that report is needed.  This
+ * entry point calls no cudaMalloc / cudaFree or allocating library routine.
+ */
+LOGO_API logo_status logo_global_attn_sparse_noalloc(const logo_bf16 *q, const logo_bf16 *k, const logo_bf16 *v,
+                                                     const float *gate, const int32_t *sel_idx, const int32_t *cu_sel,
+                                                     const logo_shape *shape, int max_selected, float scale, int merge,
+                                                     logo_bf16 *out, logo_stream_t stream);
+
+/*
  * Synchronise `stream`, then report: LOGO_ERR_CUDA if a launch or the stream
  * failed, LOGO_ERR_DEVICE_TIMEOUT if a kernel recorded a bounded wait that ran
  * out, LOGO_ERR_INVALID_ARG if a kernel recorded an argument it could not

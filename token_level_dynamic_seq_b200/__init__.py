@@ -32,7 +32,8 @@ _STATUS = {0: "LOGO_OK", 1: "LOGO_ERR_INVALID_ARG", 2: "LOGO_ERR_UNSUPPORTED", 3
 
 EXPORTED = ("logo_num_selected", "logo_workspace_size", "logo_workspace_init", "logo_select",
             "logo_local_attn", "logo_global_attn_sparse", "logo_forward", "logo_check",
-            "logo_selftest_timeout", "logo_status_string", "logo_last_error")
+            "logo_selftest_timeout", "logo_status_string", "logo_last_error",
+            "logo_global_attn_sparse_noalloc")
 
 
 class LogoError(RuntimeError):
@@ -77,6 +78,7 @@ def load_library(path: str | None = None):
             "logo_selftest_timeout": ([vp, sz, ctypes.c_uint, vp], i32),
             "logo_status_string": ([i32], ctypes.c_char_p),
             "logo_last_error": ([], ctypes.c_char_p),
+            "logo_global_attn_sparse_noalloc": ([vp, vp, vp, vp, vp, vp, sp, i32, flt, i32, vp, vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -182,6 +184,17 @@ def global_attn_sparse(q, k, v, gate, sel_idx, cu_sel, max_selected: int, out, w
     _raise(load_library().logo_global_attn_sparse(
         _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(sel_idx), _ptr(cu_sel), ctypes.byref(shape),
         int(max_selected), float(scale), 1 if merge else 0, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def global_attn_sparse_noalloc(q, k, v, gate, sel_idx, cu_sel, max_selected: int, out, scale: float = 0.0,
+                               merge: bool = True, cu_seqlens=None, max_seqlen=None, stream=None):
+    """global_attn_sparse without a caller workspace: the library's fixed scratch array is used."""
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    shape = make_shape(q, k, cu_seqlens, max_seqlen)
+    _raise(load_library().logo_global_attn_sparse_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(sel_idx), _ptr(cu_sel), ctypes.byref(shape),
+        int(max_selected), float(scale), 1 if merge else 0, _ptr(out), _stream(stream)))
     return out
 
 

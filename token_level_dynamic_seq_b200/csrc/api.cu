@@ -201,6 +201,14 @@ logo_status launch_global(const Geo& g, const void* q, const void* k, const void
 
 }  // namespace
 
+void logo::set_last_error(const char* fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+}
+
 extern "C" {
 
 int64_t logo_num_selected(double ratio, int64_t len) { return logo::budget_count(ratio, len); }

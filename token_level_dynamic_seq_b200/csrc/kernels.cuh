@@ -73,4 +73,7 @@ cudaError_t launch_timeout_probe(uint32_t* status, unsigned long long limit_ns, 
 
 size_t attn_smem_bytes(int d);
 
+// Sets the text logo_last_error() returns on this host thread.
+void set_last_error(const char* fmt, ...);
+
 }  // namespace logo
