@@ -23,7 +23,8 @@ import threading
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "liblogo.so")
+# LOGO_LIBRARY may point at another build of the same library (e.g. a tuning variant).
+LIB_PATH = os.environ.get("LOGO_LIBRARY") or os.path.join(_HERE, "liblogo.so")
 CSRC = os.path.join(_HERE, "csrc")
 
 LOGO_OK = 0

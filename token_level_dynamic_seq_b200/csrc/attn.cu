@@ -51,6 +51,16 @@ namespace {
 constexpr int kKStages = 2;
 constexpr int kVStages = 2;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
+#ifndef LOGO_POLY_EVERY
+#define LOGO_POLY_EVERY 0
+#endif
+// Every kPolyEvery-th exponential of a row uses exp2_poly (FMA pipe) instead
+// of the MUFU unit; 0 keeps them all on MUFU.
+constexpr int kPolyEvery = LOGO_POLY_EVERY;
+__device__ __forceinline__ constexpr bool use_poly(int col)
+{
+    return kPolyEvery > 0 && (col % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
+}
 
 template <int D>
 struct Geometry {
@@ -358,14 +368,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const uint32_t tS = tmem + lane_off + Geo::kTmemS + 128 * wg;
         const uint32_t tO = tmem + lane_off + Geo::kTmemO + D * wg;
-        const bool row_valid = r < w.nrows[wg];
-        const int head = w.head[wg];
+        // Per-tile fields picked with selects (no dynamic indexing into Work).
+        const int my_nrows = wg ? w.nrows[1] : w.nrows[0];
+        const int my_row0 = wg ? w.row0[1] : w.row0[0];
+        const bool row_valid = r < my_nrows;
+        const int head = wg ? w.head[1] : w.head[0];
         const int zq = w.b * p.Hq + head;
         int pos;  // position of this row within its sequence
         if (MODE == kModeLocal) {
-            pos = row_valid ? w.row0[wg] + r : w.max_pos;
+            pos = row_valid ? my_row0 + r : w.max_pos;
         } else {
-            pos = row_valid ? p.sel_idx[w.sel_base + w.row0[wg] + r] : w.max_pos;
+            pos = row_valid ? p.sel_idx[w.sel_base + my_row0 + r] : w.max_pos;
             // Gather this row of Q into the 128B-swizzled tile.
             uint8_t* dst = sQ + wg * Geo::kQBytes;
             const int4* src = reinterpret_cast<const int4*>(p.q + ((size_t)zq * p.L + w.s0 + pos) * D);
@@ -425,9 +438,34 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 m_run = m_new;
                 l_run *= alpha;
             }
+            const float mref = (m_run == -INFINITY) ? 0.f : m_run * sl2;
+            // P = exp2(S * scale * log2 e - m) in bf16 pairs; chunk c (32 columns) goes
+            // to TMEM columns 16c..16c+15 of S, whose values are already in registers.
+            float ls[8];
+            #pragma unroll
+            for (int t = 0; t < 8; ++t) ls[t] = 0.f;
+            __syncwarp();
+            #pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t pk[16];
+                #pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const int col = c * 32 + e;
+                    const float x0 = fmaf(__uint_as_float(sr[c][e]), sl2, -mref);
+                    const float x1 = fmaf(__uint_as_float(sr[c][e + 1]), sl2, -mref);
+                    // A share of the exponentials may run on the FMA pipe to unload the MUFU unit.
+                    const float p0 = use_poly(col) ? exp2_poly(x0) : fast_exp2(x0);
+                    const float p1 = use_poly(col + 1) ? exp2_poly(x1) : fast_exp2(x1);
+                    ls[(e >> 1) & 7] += p0 + p1;
+                    pk[e / 2] = pack_bf16x2(p0, p1);
+                }
+                tmem_st16(tS + c * 16, pk);
+            }
+            l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+            // Rare: the row maximum grew past the threshold, so rescale O (PV of tile
+            // j-1 is complete: see header) before this tile's PV is issued.
             const bool any = __any_sync(0xffffffffu, need);  // also reconverges the warp
             if (any && j > 0) {
-                // Rescale this warp's rows of O (PV of tile j-1 is complete: see header).
                 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t orr[32];
@@ -438,23 +476,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     tmem_st32(tO + c * 32, orr);
                 }
             }
-            const float mref = (m_run == -INFINITY) ? 0.f : m_run * sl2;
-            uint32_t pk[64];
-            float lsum = 0.f;
-            #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c][e]), sl2, -mref));
-                    const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c][e + 1]), sl2, -mref));
-                    lsum += p0 + p1;
-                    pk[c * 16 + e / 2] = pack_bf16x2(p0, p1);
-                }
-            }
-            l_run += lsum;
-            __syncwarp();
-            tmem_st32(tS, pk);
-            tmem_st32(tS + 32, pk + 32);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&p_full[wg]);

@@ -264,6 +264,32 @@ LOGO_DEVICE_INLINE float fast_exp2(float x)
     return y;
 }
 
+LOGO_DEVICE_INLINE float fmax3(float a, float b, float c)
+{
+    float y;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+    return y;
+}
+
+// 2^x for x <= 8 on the FMA pipe (no MUFU): x = n + f with n = round(x),
+// f in [-1/2, 1/2] (rounding by adding and subtracting 1.5 * 2^23), then
+// 2^x = 2^n * p(f) with p the degree-3 minimax polynomial for the relative
+// error of 2^f on [-1/2, 1/2] (max relative error 7.5e-5, derived by
+// gen_exp2_poly.py with the Remez exchange), and 2^n applied by adding n to
+// the exponent field.  x is clamped at -125 so the result stays a normal
+// number (2^-125 is far below anything that survives the bf16 P tile).
+LOGO_DEVICE_INLINE float exp2_poly(float x)
+{
+    x = fmaxf(x, -125.0f);
+    const float t = __fadd_rn(x, 12582912.0f);      // round(x) in the low mantissa bits
+    const float n = __fadd_rn(t, -12582912.0f);
+    const float f = __fadd_rn(x, -n);
+    float p = fmaf(__uint_as_float(0x3d61fbb0u), f, __uint_as_float(0x3e786f0du));
+    p = fmaf(p, f, __uint_as_float(0x3f31798du));
+    p = fmaf(p, f, __uint_as_float(0x3f7ffb49u));
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 LOGO_DEVICE_INLINE uint32_t pack_bf16x2(float lo, float hi)
 {
     uint32_t r;
