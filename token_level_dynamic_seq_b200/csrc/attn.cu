@@ -51,6 +51,13 @@ namespace {
 constexpr int kKStages = 2;
 constexpr int kVStages = 2;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
+#ifndef LOGO_P_PARTS
+#define LOGO_P_PARTS 2
+#endif
+// P_i is published in kPParts column blocks; the PV MMAs of a block start
+// while the softmax computes the next one.
+constexpr int kPParts = LOGO_P_PARTS;
+static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P is published in 1, 2 or 4 parts");
 #ifndef LOGO_POLY_EVERY
 #define LOGO_POLY_EVERY 0
 #endif
@@ -72,7 +79,7 @@ struct Geometry {
     static constexpr int kKOff = kQOff + kNumQ * kQBytes;
     static constexpr int kVOff = kKOff + kKStages * kKVBytes;
     static constexpr int kBarOff = kVOff + kVStages * kKVBytes;
-    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 3 * kNumQ + 2;
+    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + (1 + kPParts) * kNumQ + 2;
     static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
     static constexpr int kTmemS = 0;          // S_i at column 128 * i
     static constexpr int kTmemO = 128 * kNumQ; // O_i at column 256 + D * i
@@ -199,8 +206,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     uint64_t* v_full = k_empty + kKStages;
     uint64_t* v_empty = v_full + kVStages;
     uint64_t* s_full = v_empty + kVStages;
-    uint64_t* p_full = s_full + kNumQ;        // [kNumQ][2]: first / second half of P_i written
-    uint64_t* o_full = p_full + 2 * kNumQ;
+    uint64_t* p_full = s_full + kNumQ;        // [kNumQ][kPParts]: part k of P_i written
+    uint64_t* o_full = p_full + kPParts * kNumQ;
     uint64_t* drain = o_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -229,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             mbar_init(&v_empty[s], 1);
         }
         for (int i = 0; i < kNumQ; ++i) mbar_init(&s_full[i], 1);
-        for (int i = 0; i < 2 * kNumQ; ++i) mbar_init(&p_full[i], 128);
+        for (int i = 0; i < kPParts * kNumQ; ++i) mbar_init(&p_full[i], 128);
         mbar_init(o_full, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -311,12 +318,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     umma_ss(d_tmem, a, b, idesc_qk, kk > 0 ? 1u : 0u);
                 }
             };
-            // O_i += P_i V over keys 64*half .. 64*half+63 of the tile.
-            auto issue_pv = [&](int i, int vs, bool first, int half) {
+            // O_i += P_i V over the keys of P part `part` (128 / kPParts keys).
+            auto issue_pv = [&](int i, int vs, bool first, int part) {
                 const uint32_t d_tmem = tmem + Geo::kTmemO + D * i;
                 const uint32_t p_tmem = tmem + Geo::kTmemS + 128 * i;
+                constexpr int kSteps = 8 / kPParts;
                 #pragma unroll
-                for (int kk = 4 * half; kk < 4 * half + 4; ++kk) {
+                for (int kk = kSteps * part; kk < kSteps * part + kSteps; ++kk) {
                     const uint64_t b = sdesc_sw128(sVa + vs * Geo::kKVBytes + kk * 2048, Geo::kChunkBytes, 1024);
                     umma_ts(d_tmem, p_tmem + kk * 8, b, idesc_pv, (!first || kk > 0) ? 1u : 0u);
                 }
@@ -340,15 +348,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 if (!ok) break;
                 tc_fence_after();
                 for (int i = 0; i < kNumQ && ok; ++i) {
-                    // The first half of P_i is published before the second is computed.
-                    ok = mbar_wait(&p_full[2 * i], j & 1, abort_flag, p.status, limit);
+                    // P_i is published part by part while the softmax computes the rest.
+                    for (int part = 0; part < kPParts && ok; ++part) {
+                        ok = mbar_wait(&p_full[kPParts * i + part], j & 1, abort_flag, p.status, limit);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(i, vs, j == 0, part);
+                    }
                     if (!ok) break;
-                    tc_fence_after();
-                    issue_pv(i, vs, j == 0, 0);
-                    ok = mbar_wait(&p_full[2 * i + 1], j & 1, abort_flag, p.status, limit);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_pv(i, vs, j == 0, 1);
                     if (nxt) {
                         issue_s(i, ks1);
                         umma_commit(&s_full[i]);
@@ -464,32 +471,36 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 tmem_st16(tS + c * 16, pk);
             };
             __syncwarp();
-            exp_chunk(0);
-            exp_chunk(1);
-            // Rare: the row maximum grew past the threshold, so rescale O (PV of tile
-            // j-1 is complete: see header) before this tile's PV is issued.
-            const bool any = __any_sync(0xffffffffu, need);  // also reconverges the warp
-            if (any && j > 0) {
-                #pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t orr[32];
-                    tmem_ld32(tO + c * 32, orr);
-                    tmem_wait_ld(orr);
-                    #pragma unroll
-                    for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-                    tmem_st32(tO + c * 32, orr);
+            // Chunk c (32 keys) belongs to P part c / (4 / kPParts); a part is
+            // published as soon as its chunks are in TMEM.
+            #pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                exp_chunk(c);
+                if (c == 0) {
+                    // Rare: the row maximum grew past the threshold, so rescale O (PV of
+                    // tile j-1 is complete: see header) before this tile's PV is issued.
+                    const bool any = __any_sync(0xffffffffu, need);  // also reconverges the warp
+                    if (any && j > 0) {
+                        #pragma unroll 1
+                        for (int cc = 0; cc < D / 32; ++cc) {
+                            uint32_t orr[32];
+                            tmem_ld32(tO + cc * 32, orr);
+                            tmem_wait_ld(orr);
+                            #pragma unroll
+                            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                            tmem_st32(tO + cc * 32, orr);
+                        }
+                    }
+                }
+                if ((c + 1) % (4 / kPParts) == 0) {
+                    if (c == 3)
+                        l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(&p_full[kPParts * wg + c / (4 / kPParts)]);
+                    __syncwarp();
                 }
             }
-            // Publish the first half of P (keys 0..63): its PV overlaps the second half.
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&p_full[2 * wg]);
-            exp_chunk(2);
-            exp_chunk(3);
-            l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&p_full[2 * wg + 1]);
         }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, abort_flag, p.status, limit));
         if (ok) {
