@@ -10,13 +10,19 @@
 //
 // One 1024-thread CTA per sequence:
 //  1. map each fp32 logit to a 32-bit key whose unsigned order is the
-//     selection order (-0 folded onto +0, every NaN to 0, below -inf);
-//  2. radix-select the k-th largest key T with four 8-bit passes
-//     (warp-aggregated shared-memory histograms), which also yields how many
-//     keys equal to T must be taken;
-//  3. stream-compact in ascending position order with two block-wide scans
-//     per 4096-element chunk: one ranks the keys equal to T (the lowest
-//     positions win), the other places the selected positions.
+//     selection order (-0 folded onto +0, every NaN to 0, below -inf); when
+//     the sequence fits (kResidentKeys keys) the keys stay in shared memory
+//     for every later pass, otherwise each pass re-reads the logits;
+//  2. radix-select the k-th largest key T with four 8-bit passes; each warp
+//     counts into its own shared-memory histogram (no contention between
+//     warps; the lanes still matching the prefix merge equal digits with
+//     __match_any_sync, warps with no such lane skip it), and
+//     the 32 histograms are summed before the digit is chosen; this also
+//     yields how many keys equal to T must be taken;
+//  3. stream-compact in ascending position order, 4096 elements per step:
+//     a block-wide scan places the selected positions; when only some of the
+//     keys equal to T are taken, a second scan ranks those keys first (the
+//     lowest positions win).
 // Integer work only, so the result is bit-exact.
 #include <cuda_runtime.h>
 
@@ -31,6 +37,8 @@ namespace {
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kItems = 4;
+constexpr int kResidentKeys = 40960;  // 160 KB of keys kept in shared memory
+constexpr size_t kSelDynSmem = (size_t)kResidentKeys * 4 + (size_t)kSelWarps * 256 * 4;
 
 __device__ __forceinline__ uint32_t gate_key(float f)
 {
@@ -74,10 +82,14 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const float* _
                                                                   int32_t* __restrict__ sel_idx,
                                                                   int32_t* __restrict__ cu_sel)
 {
+    extern __shared__ uint32_t dyn_smem[];
+    uint32_t* keys_s = dyn_smem;                            // kResidentKeys
+    uint32_t* whist = dyn_smem + kResidentKeys;             // [kSelWarps][256]
     __shared__ uint32_t hist[256];
     __shared__ int warp_buf[32];
     __shared__ uint32_t sh_digit;
     __shared__ long long sh_remaining;
+    __shared__ uint32_t sh_bin_count;
 
     const int s = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -104,26 +116,47 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const float* _
         for (long long i = tid; i < len; i += kSelThreads) out[i] = (int32_t)i;
         return;
     }
+    const bool resident = len <= kResidentKeys;
+    if (resident) {
+        for (long long i = tid; i < len; i += kSelThreads) keys_s[i] = gate_key(__ldg(g + i));
+        __syncthreads();
+    }
+    auto key_at = [&](long long i) -> uint32_t { return resident ? keys_s[i] : gate_key(__ldg(g + i)); };
 
     // ---- radix select of the k-th largest key
     uint32_t prefix = 0, mask = 0;
     long long remaining = k;
+    uint32_t* myhist = whist + warp * 256;
     for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
-        __syncthreads();
+        for (int i = lane; i < 256; i += 32) myhist[i] = 0;
+        __syncwarp();
         for (long long base = (long long)warp * 32; base < len; base += kSelThreads) {
             const long long i = base + lane;
             const bool in = i < len;
-            const uint32_t key = in ? gate_key(g[i]) : 0u;
+            const uint32_t key = in ? key_at(i) : 0u;
             const bool match = in && ((key & mask) == prefix);
             const uint32_t digit = (key >> shift) & 255u;
-            const uint32_t tag = match ? digit : 256u + lane;  // unmatched lanes stay alone
-            const uint32_t peers = __match_any_sync(0xffffffffu, tag);
-            if (match && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (uint32_t)__popc(peers));
+            // Only lanes whose key still matches the prefix count; warps with none skip
+            // the match (its cost grows with the number of distinct values).
+            const uint32_t active = __ballot_sync(0xffffffffu, match);
+            if (match) {
+                const uint32_t peers = __match_any_sync(active, digit);
+                // one lane per distinct digit, and only this warp writes this histogram
+                if (lane == __ffs(peers) - 1) myhist[digit] += (uint32_t)__popc(peers);
+            }
+            __syncwarp();
+        }
+        __syncthreads();
+        if (tid < 256) {
+            uint32_t c = 0;
+            #pragma unroll 8
+            for (int w = 0; w < kSelWarps; ++w) c += whist[w * 256 + tid];
+            hist[tid] = c;
         }
         __syncthreads();
         if (warp == 0) {
-            // lane l owns bins 255-8l .. 248-8l (descending)
+            // lane l owns bins 255-8l .. 248-8l (descending); after the last pass the
+            // chosen bin's count is the number of keys equal to T
             uint32_t c[8];
             uint32_t sum = 0;
             #pragma unroll
@@ -145,6 +178,7 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const float* _
                     if (acc + (long long)c[t] >= remaining) {
                         sh_digit = 255u - 8u * lane - t;
                         sh_remaining = remaining - acc;
+                        sh_bin_count = c[t];
                         break;
                     }
                     acc += c[t];
@@ -155,10 +189,12 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const float* _
         prefix |= sh_digit << shift;
         mask |= 255u << shift;
         remaining = sh_remaining;
-        __syncthreads();
     }
     const uint32_t T = prefix;           // the k-th largest key
     const long long take_eq = remaining; // how many keys equal to T are selected
+    // Usually every key equal to T is taken; then "key >= T" decides alone and one
+    // scan per chunk suffices.
+    const bool all_eq = take_eq == (long long)sh_bin_count;
 
     // ---- compaction in ascending position order
     long long eq_seen = 0, written = 0;
@@ -168,11 +204,11 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const float* _
         int n_eq = 0;
         #pragma unroll
         for (int t = 0; t < kItems; ++t) {
-            keys[t] = (i0 + t < len) ? gate_key(g[i0 + t]) : 0u;
+            keys[t] = (i0 + t < len) ? key_at(i0 + t) : 0u;
             n_eq += (i0 + t < len && keys[t] == T) ? 1 : 0;
         }
-        int eq_total;
-        const int eq_before = block_exclusive_scan(n_eq, warp_buf, eq_total);
+        int eq_total = 0, eq_before = 0;
+        if (!all_eq) eq_before = block_exclusive_scan(n_eq, warp_buf, eq_total);
         bool sel[kItems];
         int n_sel = 0, eq_run = 0;
         #pragma unroll
@@ -180,7 +216,7 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const float* _
             const bool in = i0 + t < len;
             const bool gt = in && keys[t] > T;
             const bool eq = in && keys[t] == T;
-            sel[t] = gt || (eq && (eq_seen + eq_before + eq_run) < take_eq);
+            sel[t] = gt || (eq && (all_eq || (eq_seen + eq_before + eq_run) < take_eq));
             eq_run += eq ? 1 : 0;
             n_sel += sel[t] ? 1 : 0;
         }
@@ -201,7 +237,11 @@ cudaError_t launch_select(const float* gate, const int32_t* cu_seqlens, int nseq
                           int32_t* sel_idx, int32_t* cu_sel, cudaStream_t stream)
 {
     if (nseq <= 0) return cudaSuccess;
-    select_topk_kernel<<<nseq, kSelThreads, 0, stream>>>(gate, cu_seqlens, nseq, L, ratio, sel_idx, cu_sel);
+    cudaError_t e =
+        cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelDynSmem);
+    if (e != cudaSuccess) return e;
+    select_topk_kernel<<<nseq, kSelThreads, kSelDynSmem, stream>>>(gate, cu_seqlens, nseq, L, ratio, sel_idx,
+                                                                   cu_sel);
     return cudaGetLastError();
 }
 
