@@ -222,7 +222,7 @@ def main():
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
     import token_level_dynamic_seq_b200 as logo
-    from token_level_dynamic_seq_b200 import workloads
+    from token_level_dynamic_seq_b200 import multirank, workloads
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -294,11 +294,8 @@ def main():
         per["local"].append(e[1].elapsed_time(e[2]))
         per["global"].append(e[2].elapsed_time(e[3]))
     avg = {kk: sum(vv) / len(vv) for kk, vv in per.items()}
-    ms_step = t_total_ms / args.steps
-    if world > 1:
-        tt = torch.tensor([ms_step], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_step = float(tt.item())
+    ms_step = multirank.max_over_ranks(t_total_ms / args.steps, device=dev)  # slowest rank
+    job_tokens = int(multirank.sum_over_ranks(tokens, device=dev))
 
     # end to end through the public API: pinned host inputs -> forward -> host output
     pin = [x.pin_memory() for x in (w.q, w.k, w.v, w.g)]
@@ -321,11 +318,7 @@ def main():
         out_host.copy_(out, non_blocking=True)
     e2e_ev[1].record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e2e_ev[0].elapsed_time(e2e_ev[1]) / n_e2e
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = multirank.max_over_ranks(e2e_ev[0].elapsed_time(e2e_ev[1]) / n_e2e, device=dev)
     logo.check(ws, stream)
 
     peak_burst, peak_sust, hbm, peak_src = peaks()
@@ -335,7 +328,7 @@ def main():
     tr = traffic_record()
     kern_name = {"local": "attn_fwd_kernel<128, 0>", "global": "attn_fwd_kernel<128, 1>"}[dominant]
     traffic = tr.get(kern_name, {}).get("bytes_per_launch") if isinstance(tr.get(kern_name), dict) else None
-    useful_tflops = (fl_local + fl_global) / (ms_step * 1e-3) / 1e12
+    useful_tflops = multirank.sum_over_ranks(fl_local + fl_global, device=dev) / (ms_step * 1e-3) / 1e12
 
     line = None
     if rank == 0:
@@ -344,7 +337,7 @@ def main():
             cpu = cpu_baseline(w)
         line = {
             "metric": METRIC,
-            "value": tokens * world / (ms_step * 1e-3),
+            "value": job_tokens / (ms_step * 1e-3),
             "unit": "tokens/s",
             "n_gpus": world,
             "steps": args.steps,
@@ -360,7 +353,7 @@ def main():
                        "l2": "inputs larger than L2 (Q+K+V+O = %.0f MB > 126 MB)" % (
                            (q.numel() + k.numel() + v.numel() + out.numel()) * 2 / 1e6)},
             "useful_tflops": useful_tflops,
-            "useful_frac_of_bf16_peak": useful_tflops / peak_burst,
+            "useful_frac_of_bf16_peak": useful_tflops / (peak_burst * world),
             "kernels_ms": avg,
             "kernels_tflops": {"local": fl_local / (avg["local"] * 1e-3) / 1e12,
                                "global": fl_global / (avg["global"] * 1e-3) / 1e12},
@@ -368,7 +361,7 @@ def main():
             "roofline": {"kernel": kern_name, "bound": "tensor", "achieved": achieved, "peak": peak_burst,
                          "unit": "TFLOP/s", "frac": achieved / peak_burst, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16 burst (sustained {peak_sust})"},
-            "e2e": {"value": tokens * world / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": job_tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": 3 * args.steps,
             "clocks": clocks,
