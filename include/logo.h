@@ -68,7 +68,8 @@ typedef enum {
     LOGO_ERR_UNSUPPORTED = 2,    /* a shape this build does not implement (e.g. d = 96) */
     LOGO_ERR_WORKSPACE = 3,      /* workspace missing or smaller than logo_workspace_size() */
     LOGO_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed (see logo_last_error) */
-    LOGO_ERR_DEVICE_TIMEOUT = 5  /* a kernel's bounded wait ran out (read by logo_check) */
+    LOGO_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait ran out (read by logo_check) */
+    LOGO_ERR_CAPACITY = 6        /* more tokens passed a threshold than the output holds (read by logo_check) */
 } logo_status;
 
 /* Raw bf16 bit pattern. */
@@ -134,6 +135,43 @@ LOGO_API logo_status logo_workspace_init(void *ws, size_t ws_bytes, logo_stream_
  */
 LOGO_API logo_status logo_select(const float *gate, const logo_shape *shape, double ratio, int32_t *sel_idx,
                         int32_t *cu_sel, void *ws, size_t ws_bytes, logo_stream_t stream);
+
+/*
+ * Threshold form of the budget rule ("LoGo", Abstract: the budget is kept by
+ * a controller that moves a threshold on the gate, not by a fixed count).
+ * Per sequence, select the positions whose logit is strictly greater than
+ * *tau (never a NaN logit; nothing when *tau is NaN; -0 equals +0), ascending.
+ *   tau           device pointer to one fp32 threshold (e.g. kept by
+ *                 logo_threshold_update).
+ *   max_selected  per-sequence capacity; a sequence with more tokens above the
+ *                 threshold keeps its lowest max_selected positions and the
+ *                 status word records it (logo_check: LOGO_ERR_CAPACITY).
+ *   sel_idx       output, int32 (device), capacity nseq * max_selected; the
+ *                 lists of all sequences back to back.
+ *   cu_sel        output, int32 [nseq + 1] (device) offsets into sel_idx.
+ * The workspace holds the per-sequence counts (logo_workspace_size covers them).
+ * The lists feed logo_global_attn_sparse with the same max_selected.
+ */
+LOGO_API logo_status logo_select_threshold(const float *gate, const logo_shape *shape, const float *tau,
+                                           int max_selected, int32_t *sel_idx, int32_t *cu_sel, void *ws,
+                                           size_t ws_bytes, logo_stream_t stream);
+
+/*
+ * One step of the threshold controller ("LoGo", Abstract: a threshold-based
+ * controller holds the share of global tokens at a target without auxiliary
+ * losses).  Over all n logits of the batch (B * L, or cu_seqlens[nseq] when
+ * packed) with k = logo_num_selected(ratio, n), the target q is the (k+1)-th
+ * largest logit in the selection order (so, without ties, exactly k logits
+ * lie above it); q = -inf when k = n or when that place holds a NaN.  Then, in
+ * fp32 with a rounding after each operation, *tau = *tau + beta * (q - *tau),
+ * or *tau = q when either is not finite (beta = 1 jumps to the target).
+ *   tau     device pointer to one fp32 threshold, read and written.
+ *   target  device pointer receiving q, or NULL.
+ * One 1024-thread CTA runs the radix select over the whole batch.
+ */
+LOGO_API logo_status logo_threshold_update(const float *gate, const logo_shape *shape, double ratio, float beta,
+                                           float *tau, float *target, void *ws, size_t ws_bytes,
+                                           logo_stream_t stream);
 
 /*
  * Local branch for every query ("LoGo", Abstract: the windowed branch runs

@@ -53,6 +53,12 @@ def _load():
         lib.oracle_rows.argtypes = [_p, _p, _p, _p, _p, _int, _int, _int, _i64, _int, _i64, _dbl,
                                     _i64, _p, _p, _p, _p, _p, _p, _p]
         lib.oracle_rows.restype = None
+        lib.oracle_threshold_select.argtypes = [_p, _i64, ctypes.c_float, _p]
+        lib.oracle_threshold_select.restype = _i64
+        lib.oracle_threshold_target.argtypes = [_p, _i64, _dbl]
+        lib.oracle_threshold_target.restype = ctypes.c_float
+        lib.oracle_threshold_update.argtypes = [ctypes.c_float, ctypes.c_float, ctypes.c_float]
+        lib.oracle_threshold_update.restype = ctypes.c_float
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = _int
         _lib = lib
@@ -152,3 +158,22 @@ def rows(q, k, v, g, window: int, seq, head, pos, selected, scale: float = 0.0, 
                         int(window), float(scale), n, _ptr(seq_t), _ptr(head_t), _ptr(pos_t),
                         _ptr(sel_t), _ptr(loc), _ptr(glo), _ptr(out))
     return loc, glo, out
+
+
+def threshold_select(g: torch.Tensor, tau: float) -> torch.Tensor:
+    """Ascending positions of one sequence whose fp32 logit is > tau (threshold form)."""
+    g = g.detach().to(torch.float32).contiguous()
+    out = torch.empty(max(1, g.numel()), dtype=torch.int32)
+    n = _load().oracle_threshold_select(_ptr(g), g.numel(), float(tau), _ptr(out))
+    return out[:n].clone()
+
+
+def threshold_target(g: torch.Tensor, ratio: float) -> float:
+    """Target threshold: the (k+1)-th largest logit of the whole batch, k = ceil(ratio * n)."""
+    g = g.detach().to(torch.float32).contiguous().flatten()
+    return float(_load().oracle_threshold_target(_ptr(g), g.numel(), float(ratio)))
+
+
+def threshold_update(tau: float, q: float, beta: float) -> float:
+    """One controller step tau + beta * (q - tau) in fp32 (q when either is not finite)."""
+    return float(_load().oracle_threshold_update(float(tau), float(q), float(beta)))

@@ -344,6 +344,59 @@ void oracle_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, const 
     }
 }
 
+/* ---- threshold form of the budget rule -------------------------------- */
+
+/*
+ * "LoGo: Token-Level Dynamic Local-Global Attention", Abstract: the budget is
+ * kept by a controller that moves a threshold on the gate, rather than by a
+ * fixed count.  Readings used here (the pages give no formula):
+ *   selection   a token takes the global branch iff its logit is strictly
+ *               greater than the threshold tau (NaN logits never do; a NaN
+ *               tau selects nothing);
+ *   target      for n logits (the whole batch) and ratio r, with
+ *               k = oracle_num_selected(r, n), the target threshold is the
+ *               (k+1)-th largest logit in the selection order (so that, without
+ *               ties, exactly k logits lie above it); -inf when k = n; a NaN
+ *               in that place also gives -inf;
+ *   update      tau' = tau + beta * (q - tau), each operation rounded to fp32,
+ *               and tau' = q when tau or q is not finite.
+ */
+
+/* Ascending positions i < len with g[i] > tau; returns their count. */
+int64_t oracle_threshold_select(const float *g, int64_t len, float tau, int32_t *out)
+{
+    int64_t n = 0;
+    for (int64_t i = 0; i < len; ++i)
+        if (g[i] > tau) out[n++] = (int32_t)i; /* false for NaN on either side */
+    return n;
+}
+
+/* The controller's target threshold for n logits at ratio r (see above). */
+float oracle_threshold_target(const float *g, int64_t n, double ratio)
+{
+    int64_t k = oracle_num_selected(ratio, n);
+    if (k >= n) return -INFINITY;
+    gate_item *items = (gate_item *)malloc(sizeof(gate_item) * (size_t)n);
+    for (int64_t i = 0; i < n; ++i) {
+        items[i].g = g[i];
+        items[i].idx = (int32_t)i;
+    }
+    qsort(items, (size_t)n, sizeof(gate_item), gate_order);
+    float q = items[k].g; /* the (k+1)-th in the selection order */
+    free(items);
+    return isnan(q) ? -INFINITY : q;
+}
+
+/* One controller step, fp32 arithmetic with a rounding after each operation. */
+float oracle_threshold_update(float tau, float q, float beta)
+{
+    if (!isfinite(tau) || !isfinite(q)) return q;
+    volatile float diff = q - tau;
+    volatile float step = beta * diff;
+    volatile float out = tau + step;
+    return out;
+}
+
 /* Number of threads the oracle runs on (for reporting). */
 int oracle_num_threads(void)
 {

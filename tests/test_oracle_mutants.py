@@ -15,6 +15,7 @@ import pytest
 
 import oracle
 from tests import test_oracle_pins as pins
+from tests import test_oracle_threshold as tpins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "logo_oracle.c")
 
@@ -38,6 +39,10 @@ MUTANTS = {
     "denominator_dropped_term": ("den += w;", "den += (t == 0) ? 0.0 : w;"),
     "global_not_full_prefix": ("attend_row(qr, kh, vh, 0, i, p->d, p->scale, scratch, glo);",
                                "attend_row(qr, kh, vh, i > 0 ? 1 : 0, i, p->d, p->scale, scratch, glo);"),
+    "threshold_ge": ("if (g[i] > tau) out[n++] = (int32_t)i;", "if (g[i] >= tau) out[n++] = (int32_t)i;"),
+    "target_kth_not_next": ("float q = items[k].g;", "float q = items[k > 0 ? k - 1 : 0].g;"),
+    "update_drops_tau": ("volatile float out = tau + step;", "volatile float out = step;"),
+    "update_sign": ("volatile float diff = q - tau;", "volatile float diff = tau - q;"),
 }
 
 PINS = [
@@ -50,6 +55,10 @@ PINS = [
     pins.test_closed_form_uniform_weights,
     pins.test_closed_form_weights_one_e_e2,
     pins.test_ratio_one_full_window_is_gated_causal,
+    tpins.test_threshold_golden,
+    lambda: [tpins.test_threshold_select_and_target_bruteforce(s) for s in range(3)],
+    tpins.test_target_leaves_exactly_k_above_distinct_logits,
+    tpins.test_threshold_update_fp32_arithmetic,
 ]
 
 

@@ -29,12 +29,12 @@ CSRC = os.path.join(_HERE, "csrc")
 
 LOGO_OK = 0
 _STATUS = {0: "LOGO_OK", 1: "LOGO_ERR_INVALID_ARG", 2: "LOGO_ERR_UNSUPPORTED", 3: "LOGO_ERR_WORKSPACE",
-           4: "LOGO_ERR_CUDA", 5: "LOGO_ERR_DEVICE_TIMEOUT"}
+           4: "LOGO_ERR_CUDA", 5: "LOGO_ERR_DEVICE_TIMEOUT", 6: "LOGO_ERR_CAPACITY"}
 
 EXPORTED = ("logo_num_selected", "logo_workspace_size", "logo_workspace_init", "logo_select",
             "logo_local_attn", "logo_global_attn_sparse", "logo_forward", "logo_check",
             "logo_selftest_timeout", "logo_status_string", "logo_last_error",
-            "logo_global_attn_sparse_noalloc")
+            "logo_global_attn_sparse_noalloc", "logo_select_threshold", "logo_threshold_update")
 
 
 class LogoError(RuntimeError):
@@ -80,6 +80,8 @@ def load_library(path: str | None = None):
             "logo_status_string": ([i32], ctypes.c_char_p),
             "logo_last_error": ([], ctypes.c_char_p),
             "logo_global_attn_sparse_noalloc": ([vp, vp, vp, vp, vp, vp, sp, i32, flt, i32, vp, vp], i32),
+            "logo_select_threshold": ([vp, sp, vp, i32, vp, vp, vp, sz, vp], i32),
+            "logo_threshold_update": ([vp, sp, dbl, flt, vp, vp, vp, sz, vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -165,6 +167,29 @@ def select(gate: torch.Tensor, shape: Shape, ratio: float, ws: torch.Tensor, sel
     _raise(lib.logo_select(_ptr(gate), ctypes.byref(shape), float(ratio), _ptr(sel_idx), _ptr(cu_sel), _ptr(ws),
                            ws.numel(), _stream(stream)))
     return sel_idx, cu_sel
+
+
+def select_threshold(gate: torch.Tensor, shape: Shape, tau: torch.Tensor, max_selected: int, ws: torch.Tensor,
+                     sel_idx=None, cu_sel=None, stream=None):
+    """Threshold form of the budget rule: per sequence, ascending positions with logit > tau."""
+    nseq = shape.nseq if shape.cu_seqlens else shape.B
+    if sel_idx is None:
+        sel_idx = torch.empty(max(1, nseq * int(max_selected)), dtype=torch.int32, device=gate.device)
+    if cu_sel is None:
+        cu_sel = torch.empty(nseq + 1, dtype=torch.int32, device=gate.device)
+    _raise(load_library().logo_select_threshold(_ptr(gate), ctypes.byref(shape), _ptr(tau), int(max_selected),
+                                                _ptr(sel_idx), _ptr(cu_sel), _ptr(ws), ws.numel(), _stream(stream)))
+    return sel_idx, cu_sel
+
+
+def threshold_update(gate: torch.Tensor, shape: Shape, ratio: float, beta: float, tau: torch.Tensor,
+                     ws: torch.Tensor, target=None, stream=None):
+    """One controller step: moves the device threshold `tau` toward the batch target; returns target."""
+    if target is None:
+        target = torch.empty(1, dtype=torch.float32, device=gate.device)
+    _raise(load_library().logo_threshold_update(_ptr(gate), ctypes.byref(shape), float(ratio), float(beta), _ptr(tau),
+                                                _ptr(target), _ptr(ws), ws.numel(), _stream(stream)))
+    return target
 
 
 def local_attn(q, k, v, window: int, ws: torch.Tensor, scale: float = 0.0, cu_seqlens=None, max_seqlen=None,

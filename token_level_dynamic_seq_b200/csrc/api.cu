@@ -38,6 +38,9 @@ constexpr size_t kWsHeaderBytes = 256;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// After the header: per-sequence counts of the threshold selection, padded to 256 bytes.
+size_t counts_bytes(int nseq) { return ((size_t)nseq * 4 + 255) / 256 * 256; }
+
 // Geometry after validation.
 struct Geo {
     int B, Hq, Hkv, L, d, G, nseq, max_len;
@@ -217,7 +220,7 @@ size_t logo_workspace_size(const logo_shape* shape, double ratio)
 {
     Geo g;
     if (check_shape(shape, g) != LOGO_OK || check_ratio(ratio) != LOGO_OK) return 0;
-    return kWsHeaderBytes;
+    return kWsHeaderBytes + counts_bytes(g.nseq);
 }
 
 logo_status logo_workspace_init(void* ws, size_t ws_bytes, logo_stream_t stream)
@@ -318,6 +321,48 @@ logo_status logo_forward(const logo_bf16* q, const logo_bf16* k, const logo_bf16
     return launch_global(g, q, k, v, gate, sel_idx, cu_sel, max_sel, sl2, 1, out, ws, s);
 }
 
+logo_status logo_select_threshold(const float* gate, const logo_shape* shape, const float* tau, int max_selected,
+                                  int32_t* sel_idx, int32_t* cu_sel, void* ws, size_t ws_bytes, logo_stream_t stream)
+{
+    Geo g;
+    logo_status st;
+    if ((st = check_shape(shape, g)) != LOGO_OK) return st;
+    if ((st = check_ws(ws, ws_bytes)) != LOGO_OK) return st;
+    if (ws_bytes < kWsHeaderBytes + counts_bytes(g.nseq))
+        return fail(LOGO_ERR_WORKSPACE, "workspace of %zu bytes, the threshold selection needs %zu", ws_bytes,
+                    kWsHeaderBytes + counts_bytes(g.nseq));
+    if (max_selected < 0 || max_selected > g.max_len)
+        return fail(LOGO_ERR_INVALID_ARG, "max_selected=%d outside [0, %d]", max_selected, g.max_len);
+    if ((st = check_ptr(cu_sel, "cu_sel")) != LOGO_OK) return st;
+    if ((st = check_ptr(tau, "tau")) != LOGO_OK) return st;
+    if (g.L > 0 && (st = check_ptr(gate, "gate")) != LOGO_OK) return st;
+    if (max_selected > 0 && (st = check_ptr(sel_idx, "sel_idx")) != LOGO_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t* counts = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kWsHeaderBytes);
+    cudaError_t e = logo::launch_threshold_select(gate, g.cu, g.nseq, g.L, tau, max_selected, counts, sel_idx, cu_sel,
+                                                  static_cast<uint32_t*>(ws), s);
+    return e == cudaSuccess ? LOGO_OK : cuda_fail(e, "threshold select launch");
+}
+
+logo_status logo_threshold_update(const float* gate, const logo_shape* shape, double ratio, float beta, float* tau,
+                                  float* target, void* ws, size_t ws_bytes, logo_stream_t stream)
+{
+    Geo g;
+    logo_status st;
+    if ((st = check_shape(shape, g)) != LOGO_OK) return st;
+    if ((st = check_ratio(ratio)) != LOGO_OK) return st;
+    if ((st = check_ws(ws, ws_bytes)) != LOGO_OK) return st;
+    if (std::isnan(beta) || beta < 0.f || beta > 1.f) return fail(LOGO_ERR_INVALID_ARG, "beta=%g outside [0, 1]", beta);
+    if ((st = check_ptr(tau, "tau")) != LOGO_OK) return st;
+    if (target && (reinterpret_cast<uintptr_t>(target) & 3u))
+        return fail(LOGO_ERR_INVALID_ARG, "target is not 4-byte aligned");
+    if (g.L > 0 && (st = check_ptr(gate, "gate")) != LOGO_OK) return st;
+    const long long n_fixed = (long long)g.B * g.L;
+    cudaError_t e = logo::launch_threshold_update(gate, g.cu, g.nseq, n_fixed, ratio, beta, tau, target,
+                                                  static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? LOGO_OK : cuda_fail(e, "threshold update launch");
+}
+
 logo_status logo_check(const void* ws, logo_stream_t stream)
 {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
@@ -332,6 +377,8 @@ logo_status logo_check(const void* ws, logo_stream_t stream)
         return fail(LOGO_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait ran out (status 0x%x)", status);
     if (status & logo::kStatusBadArgument)
         return fail(LOGO_ERR_INVALID_ARG, "a kernel met an argument it cannot handle (status 0x%x)", status);
+    if (status & logo::kStatusCapacity)
+        return fail(LOGO_ERR_CAPACITY, "more tokens passed the threshold than max_selected (status 0x%x)", status);
     return LOGO_OK;
 }
 
@@ -355,6 +402,7 @@ const char* logo_status_string(logo_status s)
         case LOGO_ERR_WORKSPACE: return "LOGO_ERR_WORKSPACE";
         case LOGO_ERR_CUDA: return "LOGO_ERR_CUDA";
         case LOGO_ERR_DEVICE_TIMEOUT: return "LOGO_ERR_DEVICE_TIMEOUT";
+        case LOGO_ERR_CAPACITY: return "LOGO_ERR_CAPACITY";
     }
     return "LOGO_ERR_UNKNOWN";
 }

@@ -10,6 +10,7 @@ namespace logo {
 enum : uint32_t {
     kStatusTimeout = 1u,      // a bounded wait ran out
     kStatusBadArgument = 2u,  // a kernel met an argument it cannot handle
+    kStatusCapacity = 4u,     // more tokens above the threshold than the output holds
 };
 
 // Budget count, identical on host and device (see logo_num_selected in
@@ -66,6 +67,13 @@ struct alignas(64) AttnParams {
 
 cudaError_t launch_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, double ratio,
                           int32_t* sel_idx, int32_t* cu_sel, cudaStream_t stream);
+
+cudaError_t launch_threshold_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, const float* tau,
+                                    int max_selected, int32_t* counts, int32_t* sel_idx, int32_t* cu_sel,
+                                    uint32_t* status, cudaStream_t stream);
+
+cudaError_t launch_threshold_update(const float* gate, const int32_t* cu_seqlens, int nseq, long long n_fixed,
+                                    double ratio, float beta, float* tau, float* target_out, cudaStream_t stream);
 
 cudaError_t launch_attn(int mode, int d, const AttnParams& p, int max_seqlen, cudaStream_t stream);
 

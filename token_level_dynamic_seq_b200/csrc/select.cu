@@ -76,54 +76,25 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_buf, int& t
     return before + x - v;
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const float* __restrict__ gate,
-                                                                  const int32_t* __restrict__ cu_seqlens,
-                                                                  int nseq, int L, double ratio,
-                                                                  int32_t* __restrict__ sel_idx,
-                                                                  int32_t* __restrict__ cu_sel)
+struct KthResult {
+    uint32_t key;        // the k-th largest key
+    long long take_eq;   // how many keys equal to it are among the k largest
+    long long eq_count;  // how many keys equal to it there are
+};
+
+// Radix select over `len` keys (key_at(i)) with four 8-bit passes, 1 <= k <= len.
+// Called by all threads of a 1024-thread block; whist holds [kSelWarps][256]
+// per-warp histograms, hist 256 words.  Each warp counts into its own histogram
+// (the lanes still matching the prefix merge equal digits with __match_any_sync,
+// warps with no such lane skip it); the 32 histograms are summed before the
+// digit is chosen.
+template <typename KeyAt>
+__device__ KthResult radix_kth_largest(KeyAt key_at, long long len, long long k, uint32_t* whist, uint32_t* hist)
 {
-    extern __shared__ uint32_t dyn_smem[];
-    uint32_t* keys_s = dyn_smem;                            // kResidentKeys
-    uint32_t* whist = dyn_smem + kResidentKeys;             // [kSelWarps][256]
-    __shared__ uint32_t hist[256];
-    __shared__ int warp_buf[32];
     __shared__ uint32_t sh_digit;
     __shared__ long long sh_remaining;
     __shared__ uint32_t sh_bin_count;
-
-    const int s = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    long long start, len, out_off;
-    if (cu_seqlens) {
-        start = cu_seqlens[s];
-        len = (long long)cu_seqlens[s + 1] - start;
-        out_off = 0;
-        for (int t = 0; t < s; ++t) out_off += budget_count(ratio, (long long)cu_seqlens[t + 1] - cu_seqlens[t]);
-    } else {
-        start = (long long)s * L;
-        len = L;
-        out_off = (long long)s * budget_count(ratio, L);
-    }
-    const long long k = budget_count(ratio, len);
-    if (tid == 0) {
-        cu_sel[s + 1] = (int32_t)(out_off + k);
-        if (s == 0) cu_sel[0] = 0;
-    }
-    if (k <= 0) return;
-    const float* g = gate + start;
-    int32_t* out = sel_idx + out_off;
-    if (k == len) {
-        for (long long i = tid; i < len; i += kSelThreads) out[i] = (int32_t)i;
-        return;
-    }
-    const bool resident = len <= kResidentKeys;
-    if (resident) {
-        for (long long i = tid; i < len; i += kSelThreads) keys_s[i] = gate_key(__ldg(g + i));
-        __syncthreads();
-    }
-    auto key_at = [&](long long i) -> uint32_t { return resident ? keys_s[i] : gate_key(__ldg(g + i)); };
-
-    // ---- radix select of the k-th largest key
     uint32_t prefix = 0, mask = 0;
     long long remaining = k;
     uint32_t* myhist = whist + warp * 256;
@@ -136,8 +107,6 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const float* _
             const uint32_t key = in ? key_at(i) : 0u;
             const bool match = in && ((key & mask) == prefix);
             const uint32_t digit = (key >> shift) & 255u;
-            // Only lanes whose key still matches the prefix count; warps with none skip
-            // the match (its cost grows with the number of distinct values).
             const uint32_t active = __ballot_sync(0xffffffffu, match);
             if (match) {
                 const uint32_t peers = __match_any_sync(active, digit);
@@ -156,7 +125,7 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const float* _
         __syncthreads();
         if (warp == 0) {
             // lane l owns bins 255-8l .. 248-8l (descending); after the last pass the
-            // chosen bin's count is the number of keys equal to T
+            // chosen bin's count is the number of keys equal to the result
             uint32_t c[8];
             uint32_t sum = 0;
             #pragma unroll
@@ -190,11 +159,65 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const float* _
         mask |= 255u << shift;
         remaining = sh_remaining;
     }
-    const uint32_t T = prefix;           // the k-th largest key
-    const long long take_eq = remaining; // how many keys equal to T are selected
+    KthResult r;
+    r.key = prefix;
+    r.take_eq = remaining;
+    r.eq_count = (long long)sh_bin_count;
+    __syncthreads();  // the shared results may be rewritten by a later call
+    return r;
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const float* __restrict__ gate,
+                                                                  const int32_t* __restrict__ cu_seqlens,
+                                                                  int nseq, int L, double ratio,
+                                                                  int32_t* __restrict__ sel_idx,
+                                                                  int32_t* __restrict__ cu_sel)
+{
+    extern __shared__ uint32_t dyn_smem[];
+    uint32_t* keys_s = dyn_smem;                            // kResidentKeys
+    uint32_t* whist = dyn_smem + kResidentKeys;             // [kSelWarps][256]
+    __shared__ uint32_t hist[256];
+    __shared__ int warp_buf[32];
+
+    const int s = blockIdx.x;
+    const int tid = threadIdx.x;
+    long long start, len, out_off;
+    if (cu_seqlens) {
+        start = cu_seqlens[s];
+        len = (long long)cu_seqlens[s + 1] - start;
+        out_off = 0;
+        for (int t = 0; t < s; ++t) out_off += budget_count(ratio, (long long)cu_seqlens[t + 1] - cu_seqlens[t]);
+    } else {
+        start = (long long)s * L;
+        len = L;
+        out_off = (long long)s * budget_count(ratio, L);
+    }
+    const long long k = budget_count(ratio, len);
+    if (tid == 0) {
+        cu_sel[s + 1] = (int32_t)(out_off + k);
+        if (s == 0) cu_sel[0] = 0;
+    }
+    if (k <= 0) return;
+    const float* g = gate + start;
+    int32_t* out = sel_idx + out_off;
+    if (k == len) {
+        for (long long i = tid; i < len; i += kSelThreads) out[i] = (int32_t)i;
+        return;
+    }
+    const bool resident = len <= kResidentKeys;
+    if (resident) {
+        for (long long i = tid; i < len; i += kSelThreads) keys_s[i] = gate_key(__ldg(g + i));
+        __syncthreads();
+    }
+    auto key_at = [&](long long i) -> uint32_t { return resident ? keys_s[i] : gate_key(__ldg(g + i)); };
+
+    // ---- radix select of the k-th largest key
+    const KthResult kr = radix_kth_largest(key_at, len, k, whist, hist);
+    const uint32_t T = kr.key;              // the k-th largest key
+    const long long take_eq = kr.take_eq;   // how many keys equal to T are selected
     // Usually every key equal to T is taken; then "key >= T" decides alone and one
     // scan per chunk suffices.
-    const bool all_eq = take_eq == (long long)sh_bin_count;
+    const bool all_eq = take_eq == kr.eq_count;
 
     // ---- compaction in ascending position order
     long long eq_seen = 0, written = 0;
@@ -231,7 +254,156 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const float* _
     }
 }
 
+// ---------------------------------------------------------------- threshold form
+//
+// "LoGo: Token-Level Dynamic Local-Global Attention", Abstract: the budget is
+// kept by a controller that moves a threshold on the gate.  A token takes the
+// global branch iff its logit is strictly above the threshold (never for a NaN
+// logit or a NaN threshold); the comparison is done on the order-preserving
+// keys, so it is exact (-0 equals +0, no flushing of subnormals).
+
+__device__ __forceinline__ bool above(uint32_t gkey, uint32_t tkey, bool tau_nan)
+{
+    return !tau_nan && gkey > tkey;
+}
+
+__device__ __forceinline__ void seq_span(const int32_t* cu_seqlens, int L, int s, long long& start, long long& len)
+{
+    if (cu_seqlens) {
+        start = cu_seqlens[s];
+        len = (long long)cu_seqlens[s + 1] - start;
+    } else {
+        start = (long long)s * L;
+        len = L;
+    }
+}
+
+// Per sequence: how many logits lie above the threshold.
+__global__ void __launch_bounds__(kSelThreads) threshold_count_kernel(const float* __restrict__ gate,
+                                                                     const int32_t* __restrict__ cu_seqlens, int L,
+                                                                     const float* __restrict__ tau,
+                                                                     int32_t* __restrict__ counts)
+{
+    __shared__ int warp_buf[32];
+    long long start, len;
+    seq_span(cu_seqlens, L, blockIdx.x, start, len);
+    const float t = *tau;
+    const bool tau_nan = isnan(t);
+    const uint32_t tkey = gate_key(t);
+    int c = 0;
+    for (long long i = threadIdx.x; i < len; i += kSelThreads) c += above(gate_key(__ldg(gate + start + i)), tkey, tau_nan);
+    int total;
+    block_exclusive_scan(c, warp_buf, total);
+    if (threadIdx.x == 0) counts[blockIdx.x] = total;
+}
+
+// Per sequence: the positions above the threshold, ascending, at most `cap` of them,
+// written at the sequence's offset (the capped counts of the earlier sequences).
+__global__ void __launch_bounds__(kSelThreads) threshold_compact_kernel(
+    const float* __restrict__ gate, const int32_t* __restrict__ cu_seqlens, int L, const float* __restrict__ tau,
+    int cap, const int32_t* __restrict__ counts, int32_t* __restrict__ sel_idx, int32_t* __restrict__ cu_sel,
+    uint32_t* status)
+{
+    __shared__ int warp_buf[32];
+    const int s = blockIdx.x;
+    long long start, len;
+    seq_span(cu_seqlens, L, s, start, len);
+    long long off = 0;
+    for (int t = 0; t < s; ++t) off += min(counts[t], cap);
+    const int mine = min(counts[s], cap);
+    if (threadIdx.x == 0) {
+        cu_sel[s + 1] = (int32_t)(off + mine);
+        if (s == 0) cu_sel[0] = 0;
+        if (counts[s] > cap) atomicOr(status, kStatusCapacity);
+    }
+    if (mine == 0) return;
+    const float t = *tau;
+    const bool tau_nan = isnan(t);
+    const uint32_t tkey = gate_key(t);
+    int32_t* out = sel_idx + off;
+    long long written = 0;
+    for (long long chunk = 0; chunk < len && written < mine; chunk += (long long)kSelThreads * kItems) {
+        const long long i0 = chunk + (long long)threadIdx.x * kItems;
+        bool sel[kItems];
+        int n_sel = 0;
+        #pragma unroll
+        for (int u = 0; u < kItems; ++u) {
+            sel[u] = (i0 + u < len) && above(gate_key(__ldg(gate + start + i0 + u)), tkey, tau_nan);
+            n_sel += sel[u] ? 1 : 0;
+        }
+        int total;
+        const int before = block_exclusive_scan(n_sel, warp_buf, total);
+        int o = 0;
+        #pragma unroll
+        for (int u = 0; u < kItems; ++u) {
+            if (sel[u]) {
+                const long long dst = written + before + (o++);
+                if (dst < mine) out[dst] = (int32_t)(i0 + u);
+            }
+        }
+        written += total;
+    }
+}
+
+__device__ __forceinline__ float key_to_float(uint32_t key)
+{
+    if (key == 0u) return __int_as_float(0x7fc00000);  // NaN
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// The controller step over the whole batch (all n valid logits): target q = the
+// (k+1)-th largest logit, k = budget_count(ratio, n) (-inf when k = n, or when
+// that place holds a NaN); tau <- tau + beta * (q - tau) in fp32 with a rounding
+// after each operation, or tau <- q when either is not finite.
+__global__ void __launch_bounds__(kSelThreads) threshold_update_kernel(const float* __restrict__ gate,
+                                                                      const int32_t* __restrict__ cu_seqlens,
+                                                                      int nseq, long long n_fixed, double ratio,
+                                                                      float beta, float* __restrict__ tau,
+                                                                      float* __restrict__ target_out)
+{
+    extern __shared__ uint32_t dyn_smem[];
+    uint32_t* whist = dyn_smem;  // [kSelWarps][256]
+    __shared__ uint32_t hist[256];
+    const long long n = cu_seqlens ? (long long)cu_seqlens[nseq] : n_fixed;
+    const long long k = budget_count(ratio, n);
+    float q = -INFINITY;
+    if (k < n) {
+        auto key_at = [&](long long i) -> uint32_t { return gate_key(__ldg(gate + i)); };
+        const KthResult r = radix_kth_largest(key_at, n, k + 1, whist, hist);
+        q = key_to_float(r.key);
+        if (isnan(q)) q = -INFINITY;
+    }
+    if (threadIdx.x == 0) {
+        const float t = *tau;
+        const bool finite = isfinite(t) && isfinite(q);
+        *tau = finite ? __fadd_rn(t, __fmul_rn(beta, __fsub_rn(q, t))) : q;
+        if (target_out) *target_out = q;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_threshold_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, const float* tau,
+                                    int max_selected, int32_t* counts, int32_t* sel_idx, int32_t* cu_sel,
+                                    uint32_t* status, cudaStream_t stream)
+{
+    if (nseq <= 0) return cudaSuccess;
+    threshold_count_kernel<<<nseq, kSelThreads, 0, stream>>>(gate, cu_seqlens, L, tau, counts);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    threshold_compact_kernel<<<nseq, kSelThreads, 0, stream>>>(gate, cu_seqlens, L, tau, max_selected, counts,
+                                                               sel_idx, cu_sel, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_threshold_update(const float* gate, const int32_t* cu_seqlens, int nseq, long long n_fixed,
+                                    double ratio, float beta, float* tau, float* target_out, cudaStream_t stream)
+{
+    const size_t smem = (size_t)kSelWarps * 256 * 4;
+    threshold_update_kernel<<<1, kSelThreads, smem, stream>>>(gate, cu_seqlens, nseq, n_fixed, ratio, beta, tau,
+                                                              target_out);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, double ratio,
                           int32_t* sel_idx, int32_t* cu_sel, cudaStream_t stream)
