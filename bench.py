@@ -211,6 +211,66 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_decode(args, rank, world):
+    """Decode step (row f3): 64 sequences with full 32K caches, W=4096, threshold at the
+    controller target for ratio 0.2 over the 64 gate logits; HBM-bound, so the roofline is
+    the cache bytes the step must read against the measured HBM bandwidth."""
+    import token_level_dynamic_seq_b200 as logo
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    B, Hq, Hkv, L, d, W, ratio = 64, 32, 8, 32768, 128, 4096, 0.2
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(rank)
+    q = torch.randn(B, Hq, d, generator=gen, device=dev).to(torch.bfloat16)
+    kc = torch.randn(B, Hkv, L, d, generator=gen, device=dev).to(torch.bfloat16)
+    vc = torch.randn(B, Hkv, L, d, generator=gen, device=dev).to(torch.bfloat16)
+    g = torch.randn(B, generator=gen, device=dev)
+    cache_len = torch.full((B,), L, dtype=torch.int32, device=dev)
+    shape = logo.Shape(B, Hq, Hkv, L, d, None, B, L)
+    ws = logo.decode_workspace(shape, dev)
+    tau = torch.zeros(1, dtype=torch.float32, device=dev)
+    sws = logo.workspace(logo.Shape(1, 1, 1, B, d, None, 1, B), ratio, dev)
+    logo.threshold_update(g.view(1, B), logo.Shape(1, 1, 1, B, d, None, 1, B), ratio, 1.0, tau, sws)
+    out = torch.empty_like(q)
+    sel = torch.empty(B, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        logo.decode(q, kc, vc, cache_len, g, tau, W, ws=ws, out=out, selected=sel, stream=stream)
+    logo.check(ws, stream)
+    n_sel = int(sel.sum().item())
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    sampler = ClockSampler(dev.index)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    ev[0].record(stream)
+    for _ in range(args.steps):
+        logo.decode(q, kc, vc, cache_len, g, tau, W, ws=ws, out=out, selected=sel, stream=stream)
+    ev[1].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    logo.check(ws, stream)
+    ms = ev[0].elapsed_time(ev[1]) / args.steps
+    row_bytes = Hkv * d * 2 * 2  # K and V rows of all kv heads at one position
+    bytes_step = B * W * row_bytes + n_sel * (L - W) * row_bytes + 2 * B * Hq * d * 2
+    peak_burst, peak_sust, hbm, peak_src = peaks()
+    achieved = bytes_step / (ms * 1e-3) / 1e9
+    line = {
+        "metric": "LoGo decode tokens/s (64 x 32K caches, W=4096, ~20% global)", "value": B / (ms * 1e-3),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "decode_c32k", "B": B, "Hq": Hq, "Hkv": Hkv, "cache": L, "d": d, "W": W,
+                   "ratio": ratio, "selected": n_sel, "l2": "caches (8.6 GB) larger than L2"},
+        "roofline": {"kernel": "decode_partial_kernel + decode_combine_kernel", "bound": "hbm",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                     "peak_source": f"{peak_src} HBM copy bandwidth"},
+        "gpu_launches": 2 * args.steps, "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -218,6 +278,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.workload == "decode_c32k":
+        run_decode(args, rank, world)
         return
     assert args.warmup >= 3, "at least 3 warm-up steps"
 

@@ -242,6 +242,35 @@ LOGO_API logo_status logo_global_attn_sparse_noalloc(const logo_bf16 *q, const l
                                                      logo_bf16 *out, logo_stream_t stream);
 
 /*
+ * Decode step ("Learning When to Attend", "Empirical Validation and System
+ * Optimization": the gains carry over to time-to-first-token and generation;
+ * "LoGo", Abstract: per-token gate with a threshold controller).  One new
+ * query token per sequence b, at position t = cache_len[b] - 1 of its cache
+ * (its key and value already written there):
+ *   local  = softmax attention over positions max(0, t - W + 1) .. t;
+ *   global = softmax attention over 0 .. t, computed only when gate[b] > *tau
+ *            (the threshold form of the budget rule; never for NaN);
+ *   out    = local + sigmoid(gate[b]) * global, or local.
+ * Cache positions before the window are read only for tokens that take the
+ * global branch.
+ *   q        [B, Hq, d] bf16;  k_cache, v_cache [B, Hkv, Lmax, d] bf16 with
+ *            shape->L = Lmax (cu_seqlens must be NULL);  cache_len int32 [B]
+ *            (device, 0 <= cache_len <= Lmax; 0 gives a zero output; a
+ *            larger value reads nothing, gives a zero output and is reported
+ *            by logo_check as LOGO_ERR_INVALID_ARG);
+ *            gate fp32 [B];  tau one fp32 (device);  out [B, Hq, d] bf16;
+ *            selected int32 [B] (device; 1 iff gate[b] > *tau, the gate's
+ *            decision even for an empty cache) or NULL.
+ *   Hq / Hkv must be 1, 2, 4 or 8.  The workspace must hold
+ *   logo_decode_workspace_size(shape) bytes (partial softmax states).
+ */
+LOGO_API size_t logo_decode_workspace_size(const logo_shape *shape);
+LOGO_API logo_status logo_decode(const logo_bf16 *q, const logo_bf16 *k_cache, const logo_bf16 *v_cache,
+                                 const int32_t *cache_len, const float *gate, const float *tau,
+                                 const logo_shape *shape, int window, float scale, logo_bf16 *out,
+                                 int32_t *selected, void *ws, size_t ws_bytes, logo_stream_t stream);
+
+/*
  * Synchronise `stream`, then report: LOGO_ERR_CUDA if a launch or the stream
  * failed, LOGO_ERR_DEVICE_TIMEOUT if a kernel recorded a bounded wait that ran
  * out, LOGO_ERR_INVALID_ARG if a kernel recorded an argument it could not

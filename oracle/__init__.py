@@ -59,6 +59,9 @@ def _load():
         lib.oracle_threshold_target.restype = ctypes.c_float
         lib.oracle_threshold_update.argtypes = [ctypes.c_float, ctypes.c_float, ctypes.c_float]
         lib.oracle_threshold_update.restype = ctypes.c_float
+        lib.oracle_decode.argtypes = [_p, _p, _p, _p, _p, ctypes.c_float, _int, _int, _int, _i64, _int, _i64,
+                                      _dbl, _p, _p, _p, _p]
+        lib.oracle_decode.restype = _i64
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = _int
         _lib = lib
@@ -177,3 +180,21 @@ def threshold_target(g: torch.Tensor, ratio: float) -> float:
 def threshold_update(tau: float, q: float, beta: float) -> float:
     """One controller step tau + beta * (q - tau) in fp32 (q when either is not finite)."""
     return float(_load().oracle_threshold_update(float(tau), float(q), float(beta)))
+
+
+def decode(q, k_cache, v_cache, cache_len, g, tau: float, window: int, scale: float = 0.0):
+    """Decode step in fp64: q bf16 [B, Hq, d], caches bf16 [B, Hkv, Lmax, d], cache_len int32 [B]
+    (the new token at position cache_len - 1), g fp32 [B].  Returns out, local, global ([B, Hq, d]
+    fp64) and the 0/1 selection [B]."""
+    B, Hq, d = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    qb, kb, vb = _bits(q), _bits(k_cache), _bits(v_cache)
+    cl = torch.as_tensor(cache_len, dtype=torch.int32).contiguous()
+    g32 = torch.as_tensor(g, dtype=torch.float32).contiguous()
+    out = torch.empty(B, Hq, d, dtype=torch.float64)
+    loc = torch.empty_like(out)
+    glo = torch.empty_like(out)
+    sel = torch.empty(B, dtype=torch.int32)
+    _load().oracle_decode(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(cl), _ptr(g32), float(tau), B, Hq, Hkv, Lmax, d,
+                          int(window), float(scale), _ptr(out), _ptr(loc), _ptr(glo), _ptr(sel))
+    return out, loc, glo, sel

@@ -397,6 +397,76 @@ float oracle_threshold_update(float tau, float q, float beta)
     return out;
 }
 
+/* ---- decode: one new query per sequence against a key/value cache ------ */
+
+/*
+ * Decode step ("Learning When to Attend", "Empirical Validation and System
+ * Optimization": the savings carry over to time-to-first-token and
+ * generation; "LoGo", Abstract: the gate decides per token).  Readings: the
+ * new token of sequence b sits at position t = cache_len[b] - 1 of the cache
+ * (its key and value already written there); its local branch attends over
+ * positions max(0, t - W + 1) .. t; it takes the global branch iff its gate
+ * logit is strictly greater than the threshold tau (the threshold form of the
+ * budget rule), and then attends over 0 .. t; o = local + sigmoid(g) * global.
+ *   q        [B, Hq, d] bf16 bits;  k, v [B, Hkv, Lmax, d] bf16 bits.
+ *   out      [B, Hq, d] doubles;  out_local / out_global may be NULL
+ *            (out_global is 0 for tokens that do not take the global branch).
+ *   selected [B] 0/1 (may be NULL).
+ * Returns the number of tokens that took the global branch.
+ */
+int64_t oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *cache_len,
+                      const float *g, float tau, int B, int Hq, int Hkv, int64_t Lmax, int d, int64_t W,
+                      double scale, double *out, double *out_local, double *out_global, int32_t *selected)
+{
+    scale = default_scale(scale, d);
+    int G = Hq / Hkv;
+    int64_t n_sel = 0;
+    for (int b = 0; b < B; ++b) {
+        int sel = (g[b] > tau) ? 1 : 0; /* false for NaN on either side */
+        if (selected) selected[b] = sel;
+        n_sel += sel;
+    }
+    /* every (sequence, head) row is independent */
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Lmax > 0 ? Lmax : 1));
+        double *loc = (double *)malloc(sizeof(double) * (size_t)d);
+        double *glo = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t bh = 0; bh < (int64_t)B * Hq; ++bh) {
+            int b = (int)(bh / Hq), h = (int)(bh % Hq);
+            int64_t t = (int64_t)cache_len[b] - 1;
+            int sel = (g[b] > tau) ? 1 : 0;
+            double *o = out + bh * d;
+            if (t < 0) { /* empty cache: nothing to attend to */
+                for (int c = 0; c < d; ++c) {
+                    o[c] = 0.0;
+                    if (out_local) out_local[bh * d + c] = 0.0;
+                    if (out_global) out_global[bh * d + c] = 0.0;
+                }
+                continue;
+            }
+            const uint16_t *qr = q + bh * d;
+            const uint16_t *kh = k + (((int64_t)b * Hkv + h / G) * Lmax) * d;
+            const uint16_t *vh = v + (((int64_t)b * Hkv + h / G) * Lmax) * d;
+            int64_t j_lo = t - W + 1;
+            if (j_lo < 0) j_lo = 0;
+            attend_row(qr, kh, vh, j_lo, t, d, scale, s, loc);
+            if (sel) attend_row(qr, kh, vh, 0, t, d, scale, s, glo);
+            double gs = sel ? sigmoid((double)g[b]) : 0.0;
+            for (int c = 0; c < d; ++c) {
+                o[c] = loc[c] + (sel ? gs * glo[c] : 0.0);
+                if (out_local) out_local[bh * d + c] = loc[c];
+                if (out_global) out_global[bh * d + c] = sel ? glo[c] : 0.0;
+            }
+        }
+        free(s);
+        free(loc);
+        free(glo);
+    }
+    return n_sel;
+}
+
 /* Number of threads the oracle runs on (for reporting). */
 int oracle_num_threads(void)
 {

@@ -16,6 +16,7 @@ import pytest
 import oracle
 from tests import test_oracle_pins as pins
 from tests import test_oracle_threshold as tpins
+from tests import test_oracle_decode as dpins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "logo_oracle.c")
 
@@ -43,6 +44,9 @@ MUTANTS = {
     "target_kth_not_next": ("float q = items[k].g;", "float q = items[k > 0 ? k - 1 : 0].g;"),
     "update_drops_tau": ("volatile float out = tau + step;", "volatile float out = step;"),
     "update_sign": ("volatile float diff = q - tau;", "volatile float diff = tau - q;"),
+    "decode_selection_ge": ("int sel = (g[b] > tau) ? 1 : 0; /* false for NaN on either side */",
+                            "int sel = (g[b] >= tau) ? 1 : 0;"),
+    "decode_cache_last": ("int64_t t = (int64_t)cache_len[b] - 1;", "int64_t t = (int64_t)cache_len[b] - 2;"),
 }
 
 PINS = [
@@ -59,6 +63,9 @@ PINS = [
     lambda: [tpins.test_threshold_select_and_target_bruteforce(s) for s in range(3)],
     tpins.test_target_leaves_exactly_k_above_distinct_logits,
     tpins.test_threshold_update_fp32_arithmetic,
+    lambda: [dpins.test_decode_vs_dense_masks(s) for s in range(2)],
+    dpins.test_decode_matches_prefill_rows,
+    dpins.test_decode_closed_forms,
 ]
 
 

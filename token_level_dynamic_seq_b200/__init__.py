@@ -34,7 +34,8 @@ _STATUS = {0: "LOGO_OK", 1: "LOGO_ERR_INVALID_ARG", 2: "LOGO_ERR_UNSUPPORTED", 3
 EXPORTED = ("logo_num_selected", "logo_workspace_size", "logo_workspace_init", "logo_select",
             "logo_local_attn", "logo_global_attn_sparse", "logo_forward", "logo_check",
             "logo_selftest_timeout", "logo_status_string", "logo_last_error",
-            "logo_global_attn_sparse_noalloc", "logo_select_threshold", "logo_threshold_update")
+            "logo_global_attn_sparse_noalloc", "logo_select_threshold", "logo_threshold_update",
+            "logo_decode_workspace_size", "logo_decode")
 
 
 class LogoError(RuntimeError):
@@ -82,6 +83,8 @@ def load_library(path: str | None = None):
             "logo_global_attn_sparse_noalloc": ([vp, vp, vp, vp, vp, vp, sp, i32, flt, i32, vp, vp], i32),
             "logo_select_threshold": ([vp, sp, vp, i32, vp, vp, vp, sz, vp], i32),
             "logo_threshold_update": ([vp, sp, dbl, flt, vp, vp, vp, sz, vp], i32),
+            "logo_decode_workspace_size": ([sp], sz),
+            "logo_decode": ([vp, vp, vp, vp, vp, vp, sp, i32, flt, vp, vp, vp, sz, vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -190,6 +193,34 @@ def threshold_update(gate: torch.Tensor, shape: Shape, ratio: float, beta: float
     _raise(load_library().logo_threshold_update(_ptr(gate), ctypes.byref(shape), float(ratio), float(beta), _ptr(tau),
                                                 _ptr(target), _ptr(ws), ws.numel(), _stream(stream)))
     return target
+
+
+def decode_workspace(shape: Shape, device) -> torch.Tensor:
+    n = load_library().logo_decode_workspace_size(ctypes.byref(shape))
+    if n == 0:
+        _raise(1)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    _raise(load_library().logo_workspace_init(_ptr(ws), ws.numel(), _stream()))
+    return ws
+
+
+def decode(q, k_cache, v_cache, cache_len, gate, tau, window: int, ws: torch.Tensor | None = None,
+           scale: float = 0.0, out=None, selected=None, stream=None):
+    """Decode step: q [B, Hq, d], caches [B, Hkv, Lmax, d] (bf16), cache_len int32 [B], gate fp32 [B],
+    tau fp32 [1] (all CUDA).  Returns (out [B, Hq, d], selected int32 [B])."""
+    q, k_cache, v_cache = _bits(q), _bits(k_cache), _bits(v_cache)
+    B, Hq, d = q.shape
+    shape = Shape(B, Hq, k_cache.shape[1], k_cache.shape[2], d, None, B, k_cache.shape[2])
+    if ws is None:
+        ws = decode_workspace(shape, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if selected is None:
+        selected = torch.empty(B, dtype=torch.int32, device=q.device)
+    _raise(load_library().logo_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_len), _ptr(gate), _ptr(tau),
+                                      ctypes.byref(shape), int(window), float(scale), _ptr(out), _ptr(selected),
+                                      _ptr(ws), ws.numel(), _stream(stream)))
+    return out, selected
 
 
 def local_attn(q, k, v, window: int, ws: torch.Tensor, scale: float = 0.0, cu_seqlens=None, max_seqlen=None,

@@ -363,6 +363,63 @@ logo_status logo_threshold_update(const float* gate, const logo_shape* shape, do
     return e == cudaSuccess ? LOGO_OK : cuda_fail(e, "threshold update launch");
 }
 
+size_t logo_decode_workspace_size(const logo_shape* shape)
+{
+    Geo g;
+    if (check_shape(shape, g) != LOGO_OK || g.cu) return 0;
+    return kWsHeaderBytes + logo::decode_partials_bytes(g.B, g.Hkv, g.G, g.L, g.d);
+}
+
+logo_status logo_decode(const logo_bf16* q, const logo_bf16* k_cache, const logo_bf16* v_cache,
+                        const int32_t* cache_len, const float* gate, const float* tau, const logo_shape* shape,
+                        int window, float scale, logo_bf16* out, int32_t* selected, void* ws, size_t ws_bytes,
+                        logo_stream_t stream)
+{
+    Geo g;
+    logo_status st;
+    float sl2;
+    if ((st = check_shape(shape, g)) != LOGO_OK) return st;
+    if (g.cu) return fail(LOGO_ERR_INVALID_ARG, "decode takes one cache per sequence (cu_seqlens must be NULL)");
+    if (g.G != 1 && g.G != 2 && g.G != 4 && g.G != 8)
+        return fail(LOGO_ERR_UNSUPPORTED, "decode supports Hq/Hkv in {1, 2, 4, 8} (got %d)", g.G);
+    if (window < 1) return fail(LOGO_ERR_INVALID_ARG, "window=%d must be >= 1", window);
+    if ((st = resolve_scale(scale, g.d, sl2)) != LOGO_OK) return st;
+    if ((st = check_ws(ws, ws_bytes)) != LOGO_OK) return st;
+    const size_t need = kWsHeaderBytes + logo::decode_partials_bytes(g.B, g.Hkv, g.G, g.L, g.d);
+    if (ws_bytes < need) return fail(LOGO_ERR_WORKSPACE, "workspace of %zu bytes, decode needs %zu", ws_bytes, need);
+    if ((st = check_ptr(q, "q")) != LOGO_OK || (st = check_ptr(out, "out")) != LOGO_OK ||
+        (st = check_ptr(cache_len, "cache_len")) != LOGO_OK || (st = check_ptr(gate, "gate")) != LOGO_OK ||
+        (st = check_ptr(tau, "tau")) != LOGO_OK)
+        return st;
+    if (g.L > 0 && ((st = check_ptr(k_cache, "k_cache")) != LOGO_OK || (st = check_ptr(v_cache, "v_cache")) != LOGO_OK))
+        return st;
+    if (selected && (reinterpret_cast<uintptr_t>(selected) & 3u))
+        return fail(LOGO_ERR_INVALID_ARG, "selected is not 4-byte aligned");
+    logo::DecodeParams p;
+    p.q = reinterpret_cast<const uint16_t*>(q);
+    p.k = reinterpret_cast<const uint16_t*>(k_cache);
+    p.v = reinterpret_cast<const uint16_t*>(v_cache);
+    p.cache_len = cache_len;
+    p.gate = gate;
+    p.tau = tau;
+    p.out = reinterpret_cast<uint16_t*>(out);
+    p.selected = selected;
+    p.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kWsHeaderBytes);
+    p.status = static_cast<uint32_t*>(ws);
+    p.B = g.B;
+    p.Hq = g.Hq;
+    p.Hkv = g.Hkv;
+    p.G = g.G;
+    p.Lmax = g.L;
+    p.d = g.d;
+    p.W = window < g.L ? window : (g.L > 0 ? g.L : 1);
+    p.chunk = logo::kDecChunk;
+    p.nchunks = g.L > 0 ? (g.L + logo::kDecChunk - 1) / logo::kDecChunk : 1;
+    p.scale_log2 = sl2;
+    cudaError_t e = logo::launch_decode(p, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? LOGO_OK : cuda_fail(e, "decode launch");
+}
+
 logo_status logo_check(const void* ws, logo_stream_t stream)
 {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

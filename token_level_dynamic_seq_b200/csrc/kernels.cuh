@@ -75,6 +75,23 @@ cudaError_t launch_threshold_select(const float* gate, const int32_t* cu_seqlens
 cudaError_t launch_threshold_update(const float* gate, const int32_t* cu_seqlens, int nseq, long long n_fixed,
                                     double ratio, float beta, float* tau, float* target_out, cudaStream_t stream);
 
+// Decode step (decode.cu).
+constexpr int kDecChunk = 512;  // cache positions per partial CTA
+struct DecodeParams {
+    const uint16_t *q, *k, *v;  // q [B, Hq, d]; caches [B, Hkv, Lmax, d]
+    const int32_t* cache_len;   // [B]: the new token sits at cache_len - 1
+    const float* gate;          // [B]
+    const float* tau;           // one threshold (device)
+    uint16_t* out;              // [B, Hq, d]
+    int32_t* selected;          // [B] or nullptr
+    float* part;                // partial states in the workspace
+    uint32_t* status;           // workspace status word
+    int B, Hq, Hkv, G, Lmax, d, W, chunk, nchunks;
+    float scale_log2;
+};
+size_t decode_partials_bytes(int B, int Hkv, int G, int Lmax, int d);
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
+
 cudaError_t launch_attn(int mode, int d, const AttnParams& p, int max_seqlen, cudaStream_t stream);
 
 cudaError_t launch_timeout_probe(uint32_t* status, unsigned long long limit_ns, cudaStream_t stream);
