@@ -17,12 +17,14 @@
 // consecutive row tiles of one head.  Each key/value tile is staged once in
 // shared memory by TMA and feeds both query tiles.
 //
-// Warp roles (10 warps):
-//   warp 0      TMA producer: Q tiles (local mode) and the K/V ring.
-//   warp 1      tcgen05 issuer (one thread): S_i = Q_i K^T into TMEM, then
-//               O_i += P_i V with P_i read straight from TMEM.
-//   warps 2-5   softmax warpgroup for query tile 0 (thread = row = TMEM lane)
-//   warps 6-9   softmax warpgroup for query tile 1
+// Warp roles (18 warps):
+//   warp 0       TMA producer: Q tiles (local mode) and the K/V ring.
+//   warp 1       tcgen05 issuer (one thread): S_i = Q_i K^T into TMEM, then
+//                O_i += P_i V with P_i read straight from TMEM.
+//   warps 2-9    softmax for query tile 0: two warpgroups, one per half of the
+//                128 key columns (thread = row = TMEM lane); the halves meet
+//                once per tile to combine their row maxima
+//   warps 10-17  the same for query tile 1
 // TMEM (512 columns): S_0 | S_1 | O_0 | O_1.  P_i (bf16 pairs) overwrites the
 // first half of S_i once the row has been read into registers.
 //
@@ -57,13 +59,16 @@ constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 
 // P_i is published in kPParts column blocks; the PV MMAs of a block start
 // while the softmax computes the next one.
 constexpr int kPParts = LOGO_P_PARTS;
-static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P is published in 1, 2 or 4 parts");
+static_assert(kPParts == 2, "P is published in two parts, one per half-row warpgroup");
 #ifndef LOGO_POLY_EVERY
 #define LOGO_POLY_EVERY 0
 #endif
 // Every kPolyEvery-th exponential of a row uses exp2_poly (FMA pipe) instead
 // of the MUFU unit; 0 keeps them all on MUFU.
 constexpr int kPolyEvery = LOGO_POLY_EVERY;
+#ifndef LOGO_EXP_BATCH
+#define LOGO_EXP_BATCH 0
+#endif
 __device__ __forceinline__ constexpr bool use_poly(int col)
 {
     return kPolyEvery > 0 && (col % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
@@ -79,8 +84,9 @@ struct Geometry {
     static constexpr int kKOff = kQOff + kNumQ * kQBytes;
     static constexpr int kVOff = kKOff + kKStages * kKVBytes;
     static constexpr int kBarOff = kVOff + kVStages * kKVBytes;
-    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + (1 + kPParts) * kNumQ + 2;
-    static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
+    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + (2 + kPParts) * kNumQ + 2;
+    static constexpr int kXchgOff = kBarOff + kNumBars * 8 + 16;      // [kNumQ][2][128] floats
+    static constexpr int kBytes = kXchgOff + kNumQ * 2 * 128 * 4;
     static constexpr int kTmemS = 0;          // S_i at column 128 * i
     static constexpr int kTmemO = 128 * kNumQ; // O_i at column 256 + D * i
     static constexpr uint32_t kTmemCols = 512;
@@ -208,9 +214,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     uint64_t* s_full = v_empty + kVStages;
     uint64_t* p_full = s_full + kNumQ;        // [kNumQ][kPParts]: part k of P_i written
     uint64_t* o_full = p_full + kPParts * kNumQ;
-    uint64_t* drain = o_full + 1;
+    uint64_t* pair_bar = o_full + 1;          // [kNumQ]: the two halves of a row meet (256 arrivals)
+    uint64_t* drain = pair_bar + kNumQ;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    float* xchg = reinterpret_cast<float*>(smem + Geo::kXchgOff);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -226,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     if (!w.valid) return;  // uniform across the CTA
 
     if (threadIdx.x == 0) {
-        mbar_init(q_full, MODE == kModeLocal ? 1 : 128 * kNumQ);
+        mbar_init(q_full, MODE == kModeLocal ? 1 : 256 * kNumQ);
         for (int s = 0; s < kKStages; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
@@ -238,6 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         for (int i = 0; i < kNumQ; ++i) mbar_init(&s_full[i], 1);
         for (int i = 0; i < kPParts * kNumQ; ++i) mbar_init(&p_full[i], 128);
         mbar_init(o_full, 1);
+        for (int i = 0; i < kNumQ; ++i) mbar_init(&pair_bar[i], 256);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -373,12 +382,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         }
     } else {
         // ------------------------------------------------------------ softmax warpgroups
-        const int wg = (warp - 2) >> 2;          // query tile
+        // Four warpgroups: two per query tile, each owning 64 of the 128 columns
+        // of every row (thread = row = TMEM lane).  The two halves of a row meet
+        // once per tile to combine their maxima (and once at the end for the sums).
+        const int sw = (warp - 2) >> 2;          // softmax warpgroup 0..3
+        const int wg = sw >> 1;                   // query tile
+        const int half = sw & 1;                  // columns 64*half .. 64*half+63 of S_wg
         const int quarter = warp & 3;             // TMEM lane quarter this warp may touch
         const int r = quarter * 32 + lane;        // row of the tile = TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const uint32_t tS = tmem + lane_off + Geo::kTmemS + 128 * wg;
-        const uint32_t tO = tmem + lane_off + Geo::kTmemO + D * wg;
+        const uint32_t tS = tmem + lane_off + Geo::kTmemS + 128 * wg + 64 * half;  // this half's S
+        const uint32_t tP = tmem + lane_off + Geo::kTmemS + 128 * wg + 32 * half;  // this half's P
+        const uint32_t tO = tmem + lane_off + Geo::kTmemO + D * wg + (D / 2) * half;
+        float* xch = xchg + (wg * 2) * 128;       // [2][128]: one value per row from each half
+        uint64_t* pair = &pair_bar[wg];
         // Per-tile fields picked with selects (no dynamic indexing into Work).
         const int my_nrows = wg ? w.nrows[1] : w.nrows[0];
         const int my_row0 = wg ? w.row0[1] : w.row0[0];
@@ -390,16 +407,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             pos = row_valid ? my_row0 + r : w.max_pos;
         } else {
             pos = row_valid ? p.sel_idx[w.sel_base + my_row0 + r] : w.max_pos;
-            // Gather this row of Q into the 128B-swizzled tile.
+            // Gather this half of the row of Q into the 128B-swizzled tile.
             uint8_t* dst = sQ + wg * Geo::kQBytes;
             const int4* src = reinterpret_cast<const int4*>(p.q + ((size_t)zq * p.L + w.s0 + pos) * D);
+            constexpr int kUnits = Geo::kChunks * 8 / 2;  // 16-byte units per half row
             #pragma unroll
-            for (int c = 0; c < Geo::kChunks; ++c) {
-                #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    int4 val = row_valid ? __ldg(src + c * 8 + u) : make_int4(0, 0, 0, 0);
-                    *reinterpret_cast<int4*>(dst + c * Geo::kChunkBytes + r * 128 + ((u ^ (r & 7)) << 4)) = val;
-                }
+            for (int uu = 0; uu < kUnits; ++uu) {
+                const int u = half * kUnits + uu;
+                const int c = u >> 3, e = u & 7;
+                const int4 val = row_valid ? __ldg(src + u) : make_int4(0, 0, 0, 0);
+                *reinterpret_cast<int4*>(dst + c * Geo::kChunkBytes + r * 128 + ((e ^ (r & 7)) << 4)) = val;
             }
             fence_proxy_async_smem();
             mbar_arrive(q_full);
@@ -407,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const float sl2 = p.scale_log2;
         const float resc_raw = kRescaleLog2 / sl2;  // threshold in raw score units
         float m_run = -INFINITY;  // reference max (raw units)
-        float l_run = 0.f;
+        float l_run = 0.f;        // this half's share of the row sum
         bool ok = true;
         const int W = p.window;
         for (int j = 0; j < n_kv; ++j) {
@@ -415,19 +432,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], j & 1, abort_flag, p.status, limit));
             if (!ok) break;
             tc_fence_after();
-            uint32_t sr[4][32];
-            #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
-            #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_wait_ld(sr[c]);
-            const int kbase = w.kv_lo + j * kTileN;
-            const bool need_mask = (kbase + kTileN - 1 > w.min_pos) ||
-                                   (MODE == kModeLocal && kbase < w.max_pos - W + 1);
+            uint32_t sr[2][32];
+            tmem_ld32(tS, sr[0]);
+            tmem_ld32(tS + 32, sr[1]);
+            tmem_wait_ld(sr[0]);
+            tmem_wait_ld(sr[1]);
+            const int kbase = w.kv_lo + j * kTileN + 64 * half;  // position of this half's first key
+            const bool need_mask = (kbase + 63 > w.min_pos) || (MODE == kModeLocal && kbase < w.max_pos - W + 1);
             if (need_mask) {
-                const int hi = pos - kbase;                                       // keep c <= hi
-                const int lo = (MODE == kModeLocal) ? pos - W + 1 - kbase : INT_MIN; // keep c >= lo
+                const int hi = pos - kbase;                                          // keep column c <= hi
+                const int lo = (MODE == kModeLocal) ? pos - W + 1 - kbase : INT_MIN;  // keep column c >= lo
                 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 2; ++c) {
                     #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int col = c * 32 + e;
@@ -435,14 +451,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     }
                 }
             }
-            float mt = -INFINITY;
+            float mx[4];
             #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int t = 0; t < 4; ++t)
+                mx[t] = fmaxf(__uint_as_float(sr[t >> 1][(t & 1) * 16]), __uint_as_float(sr[t >> 1][(t & 1) * 16 + 1]));
+            #pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const uint32_t* rr = &sr[t >> 1][(t & 1) * 16];
                 #pragma unroll
-                for (int e = 0; e < 32; ++e) mt = fmaxf(mt, __uint_as_float(sr[c][e]));
+                for (int e = 2; e < 16; e += 2) mx[t] = fmax3(mx[t], __uint_as_float(rr[e]), __uint_as_float(rr[e + 1]));
             }
+            const float m_half = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
+            // Combine with the other half of the row.  The other half also read its S
+            // columns before arriving here, so P may overwrite them after this point.
+            xch[half * 128 + r] = m_half;
+            mbar_arrive(pair);
+            ok = __all_sync(0xffffffffu, mbar_wait(pair, j & 1, abort_flag, p.status, limit));
+            if (!ok) break;
+            const float mt = fmaxf(m_half, xch[(half ^ 1) * 128 + r]);
             const float m_new = fmaxf(m_run, mt);
-            const bool need = m_new > m_run + resc_raw;
+            const bool need = m_new > m_run + resc_raw;  // the same decision in both halves
             float alpha = 1.f;
             if (need) {
                 alpha = (m_run == -INFINITY) ? 0.f : fast_exp2((m_run - m_new) * sl2);
@@ -450,70 +478,76 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 l_run *= alpha;
             }
             const float mref = (m_run == -INFINITY) ? 0.f : m_run * sl2;
-            // P = exp2(S * scale * log2 e - m) in bf16 pairs; chunk c (32 columns) goes
-            // to TMEM columns 16c..16c+15 of S, whose values are already in registers.
-            float ls[8];
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            __syncwarp();
             #pragma unroll
-            for (int t = 0; t < 8; ++t) ls[t] = 0.f;
-            auto exp_chunk = [&](const int c) {
+            for (int c = 0; c < 2; ++c) {
                 uint32_t pk[16];
+#if LOGO_EXP_BATCH
+                // all 32 arguments, then all 32 exponentials, then packing and sums
+                float xx[32];
+                #pragma unroll
+                for (int e = 0; e < 32; ++e) xx[e] = fmaf(__uint_as_float(sr[c][e]), sl2, -mref);
+                #pragma unroll
+                for (int e = 0; e < 32; ++e) xx[e] = use_poly(64 * half + c * 32 + e) ? exp2_poly(xx[e]) : fast_exp2(xx[e]);
                 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    const int col = c * 32 + e;
+                    ls[(e >> 1) & 3] += xx[e] + xx[e + 1];
+                    pk[e / 2] = pack_bf16x2(xx[e], xx[e + 1]);
+                }
+#else
+                #pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const int col = 64 * half + c * 32 + e;
                     const float x0 = fmaf(__uint_as_float(sr[c][e]), sl2, -mref);
                     const float x1 = fmaf(__uint_as_float(sr[c][e + 1]), sl2, -mref);
                     // A share of the exponentials may run on the FMA pipe to unload the MUFU unit.
                     const float p0 = use_poly(col) ? exp2_poly(x0) : fast_exp2(x0);
                     const float p1 = use_poly(col + 1) ? exp2_poly(x1) : fast_exp2(x1);
-                    ls[(e >> 1) & 7] += p0 + p1;
+                    ls[(e >> 1) & 3] += p0 + p1;
                     pk[e / 2] = pack_bf16x2(p0, p1);
                 }
-                tmem_st16(tS + c * 16, pk);
-            };
-            __syncwarp();
-            // Chunk c (32 keys) belongs to P part c / (4 / kPParts); a part is
-            // published as soon as its chunks are in TMEM.
-            #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                exp_chunk(c);
-                if (c == 0) {
-                    // Rare: the row maximum grew past the threshold, so rescale O (PV of
-                    // tile j-1 is complete: see header) before this tile's PV is issued.
-                    const bool any = __any_sync(0xffffffffu, need);  // also reconverges the warp
-                    if (any && j > 0) {
-                        #pragma unroll 1
-                        for (int cc = 0; cc < D / 32; ++cc) {
-                            uint32_t orr[32];
-                            tmem_ld32(tO + cc * 32, orr);
-                            tmem_wait_ld(orr);
-                            #pragma unroll
-                            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-                            tmem_st32(tO + cc * 32, orr);
-                        }
-                    }
-                }
-                if ((c + 1) % (4 / kPParts) == 0) {
-                    if (c == 3)
-                        l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-                    tmem_wait_st();
-                    tc_fence_before();
-                    mbar_arrive(&p_full[kPParts * wg + c / (4 / kPParts)]);
-                    __syncwarp();
+#endif
+                tmem_st16(tP + c * 16, pk);
+            }
+            l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            // Rare: the row maximum grew past the threshold, so rescale this half's
+            // columns of O (PV of tile j-1 is complete: see header) before its PV.
+            const bool any = __any_sync(0xffffffffu, need);  // also reconverges the warp
+            if (any && j > 0) {
+                #pragma unroll 1
+                for (int c = 0; c < D / 64; ++c) {
+                    uint32_t orr[32];
+                    tmem_ld32(tO + c * 32, orr);
+                    tmem_wait_ld(orr);
+                    #pragma unroll
+                    for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                    tmem_st32(tO + c * 32, orr);
                 }
             }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&p_full[2 * wg + half]);
         }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, abort_flag, p.status, limit));
         if (ok) {
+            // Row sum: the two halves' shares.
+            xch[half * 128 + r] = l_run;
+            mbar_arrive(pair);
+            ok = __all_sync(0xffffffffu, mbar_wait(pair, n_kv & 1, abort_flag, p.status, limit));
+        }
+        if (ok) {
             tc_fence_after();
-            const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-            uint16_t* orow = p.out + ((size_t)zq * p.L + w.s0 + pos) * D;
+            const float l_row = l_run + xch[(half ^ 1) * 128 + r];
+            const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
+            uint16_t* orow = p.out + ((size_t)zq * p.L + w.s0 + pos) * D + (D / 2) * half;
             float gsig = 0.f;
             if (MODE == kModeGlobal && p.merge && row_valid) {
                 const float g = p.gate[(size_t)w.b * p.L + w.s0 + pos];
                 gsig = 1.f / (1.f + expf(-g));
             }
             #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < D / 64; ++c) {
                 uint32_t orr[32];
                 __syncwarp();
                 tmem_ld32(tO + c * 32, orr);

@@ -39,7 +39,7 @@ __host__ __device__ inline int64_t budget_count(double ratio, int64_t len)
 constexpr int kTileM = 128;   // query rows per Q tile (= TMEM lanes)
 constexpr int kTileN = 128;   // keys per K/V tile
 constexpr int kNumQ = 2;      // Q tiles per CTA, one softmax warpgroup each
-constexpr int kThreads = 64 + 128 * kNumQ;
+constexpr int kThreads = 64 + 256 * kNumQ;  // TMA warp, MMA warp, two warpgroups per query tile
 
 enum AttnMode : int { kModeLocal = 0, kModeGlobal = 1 };
 
