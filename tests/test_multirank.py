@@ -1,10 +1,11 @@
 """Multi-rank host logic on the CPU (gloo, world size 2).
 
-The forward pass splits across ranks by whole sequences with no exchange on
-the data path.  These tests check the assignment (every sequence exactly
-once, balanced by attention cost), the per-rank packing, and that two gloo
-ranks each running their own share reproduce the single-process result row
-for row (with the fp64 oracle standing in for the GPU kernels, which the CPU
+The forward pass splits across ranks by whole sequences, or by whole
+key/value-head groups, with no exchange on the data path.  These tests check
+the assignment (every sequence exactly once, balanced by attention cost; every
+head exactly once, in whole groups), the per-rank packing, and that two gloo
+ranks each running their own share reproduce the single-process result
+element for element (with the fp64 oracle standing in for the GPU kernels, which the CPU
 box does not have).  The max / sum reductions used for whole-job timing are
 checked on the same two ranks.
 """
@@ -97,3 +98,46 @@ def test_two_gloo_ranks_reproduce_single_process(tmp_path):
     assert r["max"] == 2.0
     assert r["sum"] == float(sum(w.seqlens))
     assert all(len(sh) > 0 for sh in r["shards"])
+
+
+def test_shard_heads_whole_groups():
+    for Hq, Hkv in ((32, 8), (8, 8), (6, 2), (4, 1)):
+        for world in (1, 2, 3, 4, 8):
+            shards = multirank.shard_heads(Hq, Hkv, world)
+            G = Hq // Hkv
+            covered = []
+            for h0, h1, hk0, hk1 in shards:
+                assert h0 == hk0 * G and h1 == hk1 * G
+                covered += list(range(h0, h1))
+            assert covered == list(range(Hq))
+
+
+def _head_rank_main(rank, world, port, out_path):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = workloads.make(1, 8, 4, 45, 16, 9, 0.25, seed=5, qkv_scale=1.0)
+        shard = multirank.shard_heads(w.Hq, w.Hkv, world)[rank]
+        q, k, v = multirank.head_slice(w.q, w.k, w.v, shard)
+        res = oracle.forward(q, k, v, w.g, w.W, w.ratio)
+        gathered = [None] * world
+        dist.all_gather_object(gathered, (shard, res["out"], res["sel_idx"].tolist()))
+        if rank == 0:
+            with open(out_path, "wb") as f:
+                pickle.dump(gathered, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_head_shards_reproduce_single_process(tmp_path):
+    out_path = str(tmp_path / "heads.pkl")
+    mp.spawn(_head_rank_main, args=(2, _free_port(), out_path), nprocs=2, join=True)
+    with open(out_path, "rb") as f:
+        gathered = pickle.load(f)
+    w = workloads.make(1, 8, 4, 45, 16, 9, 0.25, seed=5, qkv_scale=1.0)
+    full = oracle.forward(w.q, w.k, w.v, w.g, w.W, w.ratio)
+    for (h0, h1, _, _), out, sel in gathered:
+        assert sel == full["sel_idx"].tolist()  # every rank recomputes the same selection
+        assert torch.equal(out, full["out"][:, h0:h1])

@@ -1,13 +1,17 @@
 """Splitting the forward pass across ranks (one process per GPU).
 
-The forward pass partitions into independent problems: the sequences of a
-batch never attend to one another ("Local-global attention", Implementation
-sketch notes, "Packed examples (LongT5)"), and the budget is per sequence, so
-each rank can run whole sequences with no exchange on the data path.  This
-module holds the host logic for that: a longest-processing-time assignment of
-sequences to ranks by their attention cost, the packing of a rank's
-sequences into its own varlen batch, and the max / sum reductions used to
-report whole-job timings.  No collective touches the attention data.
+The forward pass partitions into independent problems, two ways:
+  * by sequence: the sequences of a batch never attend to one another
+    ("Local-global attention", Implementation sketch notes, "Packed examples
+    (LongT5)") and the budget is per sequence;
+  * by head: every head attends on its own, and the selection depends only on
+    the gate logits, which every rank holds whole (they are tiny), so each rank
+    runs its key/value-head groups and recomputes the same selection.
+Either way no collective touches the attention data.  This module holds the
+host logic for both: a longest-processing-time assignment of sequences to
+ranks by their attention cost, the packing of a rank's sequences into its own
+varlen batch, the split of heads in whole key/value groups, and the max / sum
+reductions used to report whole-job timings.
 """
 from __future__ import annotations
 
@@ -88,3 +92,25 @@ def sum_over_ranks(value: float, device=None) -> float:
     """Sum over all ranks (e.g. tokens processed by the whole job)."""
     import torch.distributed as dist
     return _reduce(value, dist.ReduceOp.SUM, device)
+
+
+def shard_heads(Hq: int, Hkv: int, world: int) -> list[tuple[int, int, int, int]]:
+    """Split the query heads over ranks in whole key/value groups (GQA: query head h
+    reads key/value head h / (Hq / Hkv)), so a rank needs only its own K/V heads and no
+    exchange on the data path.  Returns per rank (h0, h1, hk0, hk1): query heads
+    [h0, h1) and key/value heads [hk0, hk1); ranks beyond Hkv get empty ranges."""
+    if world < 1 or Hkv < 1 or Hq % Hkv:
+        raise ValueError("need world >= 1 and Hq a multiple of Hkv")
+    G = Hq // Hkv
+    out = []
+    for r in range(world):
+        hk0 = (Hkv * r) // world
+        hk1 = (Hkv * (r + 1)) // world
+        out.append((hk0 * G, hk1 * G, hk0, hk1))
+    return out
+
+
+def head_slice(q, k, v, shard):
+    """The rank's share of [B, H, L, d] tensors for one shard from shard_heads."""
+    h0, h1, hk0, hk1 = shard
+    return q[:, h0:h1].contiguous(), k[:, hk0:hk1].contiguous(), v[:, hk0:hk1].contiguous()
