@@ -62,6 +62,12 @@ def _load():
         lib.oracle_decode.argtypes = [_p, _p, _p, _p, _p, ctypes.c_float, _int, _int, _int, _i64, _int, _i64,
                                       _dbl, _p, _p, _p, _p]
         lib.oracle_decode.restype = _i64
+        lib.oracle_backward.argtypes = [_p, _p, _p, _p, _p, _p, _int, _int, _int, _i64, _int, _i64, _dbl, _dbl,
+                                        _p, _p, _p, _p]
+        lib.oracle_backward.restype = _i64
+        lib.oracle_backward_rows.argtypes = [_p, _p, _p, _p, _p, _p, _p, _int, _int, _int, _i64, _int, _i64, _dbl,
+                                             _i64, _p, _p, _p, _p, _p, _i64, _p, _p, _p, _p, _p]
+        lib.oracle_backward_rows.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = _int
         _lib = lib
@@ -198,3 +204,70 @@ def decode(q, k_cache, v_cache, cache_len, g, tau: float, window: int, scale: fl
     _load().oracle_decode(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(cl), _ptr(g32), float(tau), B, Hq, Hkv, Lmax, d,
                           int(window), float(scale), _ptr(out), _ptr(loc), _ptr(glo), _ptr(sel))
     return out, loc, glo, sel
+
+
+def backward(q, k, v, g, dout, window: int, ratio: float, scale: float = 0.0, cu_seqlens=None):
+    """Whole backward pass in fp64 (chain rule through :func:`forward`).
+
+    ``dout`` is bf16 with the shape of the output.  Returns a dict with
+    ``dq`` [B, Hq, L, d], ``dk``, ``dv`` [B, Hkv, L, d] and ``dg`` [B, L]
+    (fp64), and the number of selected tokens ``n_sel``.
+    """
+    B, Hq, Hkv, L, d, nseq = _geometry(q, k, cu_seqlens)
+    qb, kb, vb, eb = _bits(q), _bits(k), _bits(v), _bits(dout)
+    g32 = g.detach().to(torch.float32).contiguous()
+    cu = None if cu_seqlens is None else cu_seqlens.to(torch.int32).contiguous()
+    dq = torch.empty(B, Hq, L, d, dtype=torch.float64)
+    dk = torch.empty(B, Hkv, L, d, dtype=torch.float64)
+    dv = torch.empty_like(dk)
+    dg = torch.empty(B, L, dtype=torch.float64)
+    n = _load().oracle_backward(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(g32), _ptr(eb), _ptr(cu), nseq, Hq, Hkv, L, d,
+                                int(window), float(ratio), float(scale), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg))
+    return {"dq": dq, "dk": dk, "dv": dv, "dg": dg, "n_sel": int(n)}
+
+
+def selection_flags(g, ratio: float, cu_seqlens=None) -> torch.Tensor:
+    """uint8 [B, L]: 1 where the budget rule selects the position (per sequence)."""
+    g32 = g.detach().to(torch.float32)
+    B, L = g32.shape
+    flags = torch.zeros(B, L, dtype=torch.uint8)
+    if cu_seqlens is None:
+        spans = [(b, 0, L) for b in range(B)]
+    else:
+        cu = cu_seqlens.tolist()
+        spans = [(0, cu[s], cu[s + 1]) for s in range(len(cu) - 1)]
+    for b, a, e in spans:
+        if e > a:
+            flags[b, a + select(g32[b, a:e], ratio).long()] = 1
+    return flags
+
+
+def backward_rows(q, k, v, g, dout, window: int, ratio: float, qrows=(), krows=(), scale: float = 0.0,
+                  cu_seqlens=None, flags=None):
+    """Sampled gradient rows in fp64.
+
+    ``qrows``: (seq, query head, position) triples -> ``dq`` [nq, d] and the
+    gate gradient ``dg`` [nq] at that position (all heads).  ``krows``:
+    (seq, key/value head, position) -> ``dk``, ``dv`` [nk, d].  Positions are
+    relative to the sequence start.
+    """
+    B, Hq, Hkv, L, d, nseq = _geometry(q, k, cu_seqlens)
+    qb, kb, vb, eb = _bits(q), _bits(k), _bits(v), _bits(dout)
+    g32 = g.detach().to(torch.float32).contiguous()
+    cu = None if cu_seqlens is None else cu_seqlens.to(torch.int32).contiguous()
+    if flags is None:
+        flags = selection_flags(g32, ratio, cu)
+    flags = flags.to(torch.uint8).contiguous()
+    qr = list(qrows)
+    kr = list(krows)
+    cols = lambda rows, i, dt: torch.tensor([r[i] for r in rows] or [0], dtype=dt)
+    qs, qh, qp = cols(qr, 0, torch.int32), cols(qr, 1, torch.int32), cols(qr, 2, torch.int64)
+    ks, kh, kp = cols(kr, 0, torch.int32), cols(kr, 1, torch.int32), cols(kr, 2, torch.int64)
+    dq = torch.empty(max(1, len(qr)), d, dtype=torch.float64)
+    dg = torch.empty(max(1, len(qr)), dtype=torch.float64)
+    dk = torch.empty(max(1, len(kr)), d, dtype=torch.float64)
+    dv = torch.empty_like(dk)
+    _load().oracle_backward_rows(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(g32), _ptr(eb), _ptr(flags), _ptr(cu), nseq,
+                                 Hq, Hkv, L, d, int(window), float(scale), len(qr), _ptr(qs), _ptr(qh), _ptr(qp),
+                                 _ptr(dq), _ptr(dg), len(kr), _ptr(ks), _ptr(kh), _ptr(kp), _ptr(dk), _ptr(dv))
+    return {"dq": dq[:len(qr)], "dg": dg[:len(qr)], "dk": dk[:len(kr)], "dv": dv[:len(kr)]}

@@ -476,3 +476,260 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* ---- backward pass ---------------------------------------------------- */
+
+/*
+ * Gradients of a scalar loss through the forward pass above, given the
+ * loss's gradient with respect to the merged output ("dout").  The pages
+ * print no backward formulas; they say the method is trained end to end and
+ * that its kernels speed up training ("Learning When to Attend", "Empirical
+ * Validation and System Optimization"; "LoGo", Abstract: a learned gate with
+ * no auxiliary loss).  What follows is the chain rule through the forward
+ * definition, with one reading:
+ *   gate        o_i depends on g_i only through the factor sigmoid(g_i) on
+ *               selected rows; the selection itself is a step function of the
+ *               logits and passes no gradient.  So
+ *               dL/dg_i = sigmoid(g_i) (1 - sigmoid(g_i)) sum_h <dout_hi, global_hi>
+ *               for selected i, 0 otherwise.
+ * For one softmax row with probabilities P_j over its keys, output
+ * o = sum_j P_j v_j and upstream gradient e (dout for the local branch,
+ * sigmoid(g_i) dout for the global branch):
+ *   dv_j += P_j e;  dP_j = <e, v_j>;  D = <e, o>;  dS_j = P_j (dP_j - D);
+ *   dq += scale sum_j dS_j k_j;  dk_j += scale dS_j q.
+ * Key/value gradients sum over the query heads of a GQA group.
+ */
+
+/* The probabilities of one softmax row (keys j_lo..j_hi) into p[], its output into o[]. */
+static void row_probs(const uint16_t *q, const uint16_t *kh, const uint16_t *vh, int64_t j_lo,
+                      int64_t j_hi, int d, double scale, double *p, double *o)
+{
+    int64_t n = j_hi - j_lo + 1;
+    double m = -INFINITY;
+    for (int64_t t = 0; t < n; ++t) {
+        const uint16_t *kr = kh + (int64_t)d * (j_lo + t);
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c) dot += bf16_bits_to_double(q[c]) * bf16_bits_to_double(kr[c]);
+        p[t] = scale * dot;
+        if (p[t] > m) m = p[t];
+    }
+    double den = 0.0;
+    for (int64_t t = 0; t < n; ++t) {
+        p[t] = exp(p[t] - m);
+        den += p[t];
+    }
+    for (int c = 0; c < d; ++c) o[c] = 0.0;
+    for (int64_t t = 0; t < n; ++t) {
+        p[t] /= den;
+        const uint16_t *vr = vh + (int64_t)d * (j_lo + t);
+        for (int c = 0; c < d; ++c) o[c] += p[t] * bf16_bits_to_double(vr[c]);
+    }
+}
+
+/*
+ * Backward of one softmax row with upstream gradient e = a * dout (a = 1 for
+ * the local branch, sigmoid(g_i) for the global one).  p[] and o[] come from
+ * row_probs.  Adds into dq (d doubles, may be NULL) and into the key/value
+ * gradient rows dk[j], dv[j] (rows d apart, indexed from the sequence start;
+ * may be NULL).  If only_key >= 0, only key j = only_key takes its dk/dv share.
+ */
+static void row_grad(const uint16_t *q, const uint16_t *kh, const uint16_t *vh, const uint16_t *dout,
+                     double a, int64_t j_lo, int64_t j_hi, int d, double scale, const double *p,
+                     const double *o, double *dq, double *dk, double *dv, int64_t only_key)
+{
+    double D = 0.0;
+    for (int c = 0; c < d; ++c) D += a * bf16_bits_to_double(dout[c]) * o[c];
+    for (int64_t j = j_lo; j <= j_hi; ++j) {
+        if (!dq && only_key >= 0 && j != only_key) continue;
+        const uint16_t *kr = kh + j * (int64_t)d;
+        const uint16_t *vr = vh + j * (int64_t)d;
+        double pj = p[j - j_lo];
+        double dp = 0.0;
+        for (int c = 0; c < d; ++c) dp += a * bf16_bits_to_double(dout[c]) * bf16_bits_to_double(vr[c]);
+        double ds = pj * (dp - D);
+        if (dq)
+            for (int c = 0; c < d; ++c) dq[c] += scale * ds * bf16_bits_to_double(kr[c]);
+        if (only_key >= 0 && j != only_key) continue;
+        double *dkr = dk ? dk + (only_key >= 0 ? 0 : j * (int64_t)d) : NULL;
+        double *dvr = dv ? dv + (only_key >= 0 ? 0 : j * (int64_t)d) : NULL;
+        for (int c = 0; c < d; ++c) {
+            if (dkr) dkr[c] += scale * ds * bf16_bits_to_double(q[c]);
+            if (dvr) dvr[c] += pj * a * bf16_bits_to_double(dout[c]);
+        }
+    }
+}
+
+/*
+ * Full backward pass.  Inputs as for oracle_forward, plus dout [B, Hq, L, d]
+ * bf16 bits.  Outputs (doubles, overwritten): dq [B, Hq, L, d],
+ * dk and dv [B, Hkv, L, d], dg [B, L] (0 on rows outside every sequence).
+ * Returns the total number of selected tokens.
+ */
+int64_t oracle_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                        const uint16_t *dout, const int32_t *cu_seqlens, int nseq, int Hq, int Hkv, int64_t L,
+                        int d, int64_t W, double ratio, double scale, double *dq, double *dk, double *dv,
+                        double *dg)
+{
+    problem pr = {q, k, v, g, cu_seqlens, nseq, Hq, Hkv, d, L, W, default_scale(scale, d)};
+    int64_t B = cu_seqlens ? 1 : nseq;
+    int G = Hq / Hkv;
+    memset(dq, 0, sizeof(double) * (size_t)(B * Hq * L * d));
+    memset(dk, 0, sizeof(double) * (size_t)(B * Hkv * L * d));
+    memset(dv, 0, sizeof(double) * (size_t)(B * Hkv * L * d));
+    memset(dg, 0, sizeof(double) * (size_t)(B * L));
+    int64_t total = 0;
+    for (int s = 0; s < nseq; ++s) {
+        int64_t b = cu_seqlens ? 0 : s;
+        int64_t s0 = seq_start(&pr, s), len = seq_len(&pr, s);
+        if (len <= 0) continue;
+        unsigned char *flag = (unsigned char *)calloc((size_t)len, 1);
+        int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)len);
+        int64_t ks = oracle_select(g + b * L + s0, len, ratio, sel);
+        for (int64_t t = 0; t < ks; ++t) flag[sel[t]] = 1;
+        total += ks;
+        /* per row and head: <dout, global>, for the gate gradient */
+        double *gdot = (double *)calloc((size_t)(len * Hq), sizeof(double));
+        /* key/value heads are independent; the query heads of a group share dk, dv */
+#pragma omp parallel
+        {
+            double *p = (double *)malloc(sizeof(double) * (size_t)len);
+            double *o = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 1)
+            for (int hk = 0; hk < Hkv; ++hk) {
+                const uint16_t *kh = row_ptr(k, b, Hkv, hk, L, s0, d);
+                const uint16_t *vh = row_ptr(v, b, Hkv, hk, L, s0, d);
+                double *dkh = dk + ((b * Hkv + hk) * L + s0) * (int64_t)d;
+                double *dvh = dv + ((b * Hkv + hk) * L + s0) * (int64_t)d;
+                for (int h = hk * G; h < (hk + 1) * G; ++h) {
+                    for (int64_t i = 0; i < len; ++i) {
+                        const uint16_t *qr = row_ptr(q, b, Hq, h, L, s0 + i, d);
+                        const uint16_t *er = row_ptr(dout, b, Hq, h, L, s0 + i, d);
+                        double *dqr = dq + ((b * Hq + h) * L + s0 + i) * (int64_t)d;
+                        int64_t j_lo = i - W + 1;
+                        if (j_lo < 0) j_lo = 0;
+                        row_probs(qr, kh, vh, j_lo, i, d, pr.scale, p, o);
+                        row_grad(qr, kh, vh, er, 1.0, j_lo, i, d, pr.scale, p, o, dqr, dkh, dvh, -1);
+                        if (flag[i]) {
+                            double a = sigmoid((double)g[b * L + s0 + i]);
+                            row_probs(qr, kh, vh, 0, i, d, pr.scale, p, o);
+                            row_grad(qr, kh, vh, er, a, 0, i, d, pr.scale, p, o, dqr, dkh, dvh, -1);
+                            double e = 0.0;
+                            for (int c = 0; c < d; ++c) e += bf16_bits_to_double(er[c]) * o[c];
+                            gdot[i * Hq + h] = e;
+                        }
+                    }
+                }
+            }
+            free(p);
+            free(o);
+        }
+        for (int64_t i = 0; i < len; ++i) {
+            if (!flag[i]) continue;
+            double sg = sigmoid((double)g[b * L + s0 + i]);
+            double e = 0.0;
+            for (int h = 0; h < Hq; ++h) e += gdot[i * Hq + h];
+            dg[b * L + s0 + i] = sg * (1.0 - sg) * e;
+        }
+        free(gdot);
+        free(sel);
+        free(flag);
+    }
+    return total;
+}
+
+/*
+ * Sampled gradient rows, for problems too large to run whole.  `flags` holds
+ * one byte per row of the [B, L] gate (1 = selected; from oracle_select).
+ *   Query rows t < nq: (qseq[t], qhead[t], qpos[t]) -> dq_out[t*d ..] and,
+ *   summed over all heads at that position, dg_out[t].
+ *   Key rows t < nk: (kseq[t], khead[t] = key/value head, kpos[t]) ->
+ *   dk_out[t*d ..], dv_out[t*d ..]: the shares of every query row (local
+ *   window and selected rows) of every query head of the group that reads it.
+ * Positions are relative to the sequence start.
+ */
+void oracle_backward_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                          const uint16_t *dout, const unsigned char *flags, const int32_t *cu_seqlens, int nseq,
+                          int Hq, int Hkv, int64_t L, int d, int64_t W, double scale, int64_t nq,
+                          const int32_t *qseq, const int32_t *qhead, const int64_t *qpos, double *dq_out,
+                          double *dg_out, int64_t nk, const int32_t *kseq, const int32_t *khead,
+                          const int64_t *kpos, double *dk_out, double *dv_out)
+{
+    problem pr = {q, k, v, g, cu_seqlens, nseq, Hq, Hkv, d, L, W, default_scale(scale, d)};
+    int G = Hq / Hkv;
+    int64_t maxlen = 1;
+    for (int s = 0; s < nseq; ++s)
+        if (seq_len(&pr, s) > maxlen) maxlen = seq_len(&pr, s);
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (size_t)maxlen);
+        double *o = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < nq + nk; ++t) {
+            int is_q = t < nq;
+            int64_t u = is_q ? t : t - nq;
+            int s = is_q ? qseq[u] : kseq[u];
+            int64_t b = cu_seqlens ? 0 : s;
+            int64_t s0 = seq_start(&pr, s), len = seq_len(&pr, s);
+            if (is_q) {
+                int h = qhead[u];
+                int64_t i = qpos[u];
+                const uint16_t *kh = row_ptr(k, b, Hkv, h / G, L, s0, d);
+                const uint16_t *vh = row_ptr(v, b, Hkv, h / G, L, s0, d);
+                double *dqr = dq_out + u * d;
+                for (int c = 0; c < d; ++c) dqr[c] = 0.0;
+                int64_t j_lo = i - W + 1;
+                if (j_lo < 0) j_lo = 0;
+                const uint16_t *qr = row_ptr(q, b, Hq, h, L, s0 + i, d);
+                const uint16_t *er = row_ptr(dout, b, Hq, h, L, s0 + i, d);
+                row_probs(qr, kh, vh, j_lo, i, d, pr.scale, p, o);
+                row_grad(qr, kh, vh, er, 1.0, j_lo, i, d, pr.scale, p, o, dqr, NULL, NULL, -1);
+                double e = 0.0;
+                if (flags[b * L + s0 + i]) {
+                    double sg = sigmoid((double)g[b * L + s0 + i]);
+                    row_probs(qr, kh, vh, 0, i, d, pr.scale, p, o);
+                    row_grad(qr, kh, vh, er, sg, 0, i, d, pr.scale, p, o, dqr, NULL, NULL, -1);
+                    /* the gate: every head at this position */
+                    for (int hh = 0; hh < Hq; ++hh) {
+                        const uint16_t *q2 = row_ptr(q, b, Hq, hh, L, s0 + i, d);
+                        const uint16_t *e2 = row_ptr(dout, b, Hq, hh, L, s0 + i, d);
+                        const uint16_t *k2 = row_ptr(k, b, Hkv, hh / G, L, s0, d);
+                        const uint16_t *v2 = row_ptr(v, b, Hkv, hh / G, L, s0, d);
+                        row_probs(q2, k2, v2, 0, i, d, pr.scale, p, o);
+                        for (int c = 0; c < d; ++c) e += bf16_bits_to_double(e2[c]) * o[c];
+                    }
+                    e *= sg * (1.0 - sg);
+                }
+                if (dg_out) dg_out[u] = e;
+            } else {
+                int hk = khead[u];
+                int64_t j = kpos[u];
+                const uint16_t *kh = row_ptr(k, b, Hkv, hk, L, s0, d);
+                const uint16_t *vh = row_ptr(v, b, Hkv, hk, L, s0, d);
+                double *dkr = dk_out + u * d, *dvr = dv_out + u * d;
+                for (int c = 0; c < d; ++c) dkr[c] = dvr[c] = 0.0;
+                for (int h = hk * G; h < (hk + 1) * G; ++h) {
+                    for (int64_t i = j; i < len; ++i) {
+                        int local = i - j < W;
+                        int glob = flags[b * L + s0 + i] != 0;
+                        if (!local && !glob) continue;
+                        const uint16_t *qr = row_ptr(q, b, Hq, h, L, s0 + i, d);
+                        const uint16_t *er = row_ptr(dout, b, Hq, h, L, s0 + i, d);
+                        if (local) {
+                            int64_t j_lo = i - W + 1;
+                            if (j_lo < 0) j_lo = 0;
+                            row_probs(qr, kh, vh, j_lo, i, d, pr.scale, p, o);
+                            row_grad(qr, kh, vh, er, 1.0, j_lo, i, d, pr.scale, p, o, NULL, dkr, dvr, j);
+                        }
+                        if (glob) {
+                            double sg = sigmoid((double)g[b * L + s0 + i]);
+                            row_probs(qr, kh, vh, 0, i, d, pr.scale, p, o);
+                            row_grad(qr, kh, vh, er, sg, 0, i, d, pr.scale, p, o, NULL, dkr, dvr, j);
+                        }
+                    }
+                }
+            }
+        }
+        free(p);
+        free(o);
+    }
+}

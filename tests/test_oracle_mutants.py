@@ -17,6 +17,7 @@ import oracle
 from tests import test_oracle_pins as pins
 from tests import test_oracle_threshold as tpins
 from tests import test_oracle_decode as dpins
+from tests import test_oracle_backward as bpins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "logo_oracle.c")
 
@@ -47,6 +48,23 @@ MUTANTS = {
     "decode_selection_ge": ("int sel = (g[b] > tau) ? 1 : 0; /* false for NaN on either side */",
                             "int sel = (g[b] >= tau) ? 1 : 0;"),
     "decode_cache_last": ("int64_t t = (int64_t)cache_len[b] - 1;", "int64_t t = (int64_t)cache_len[b] - 2;"),
+    "bwd_drop_D": ("double ds = pj * (dp - D);", "double ds = pj * dp;"),
+    "bwd_gate_no_derivative": ("dg[b * L + s0 + i] = sg * (1.0 - sg) * e;", "dg[b * L + s0 + i] = sg * e;"),
+    "bwd_global_upstream_ungated": (
+        "row_grad(qr, kh, vh, er, a, 0, i, d, pr.scale, p, o, dqr, dkh, dvh, -1);",
+        "row_grad(qr, kh, vh, er, 1.0, 0, i, d, pr.scale, p, o, dqr, dkh, dvh, -1);"),
+    "bwd_dk_unscaled": ("if (dkr) dkr[c] += scale * ds * bf16_bits_to_double(q[c]);",
+                        "if (dkr) dkr[c] += ds * bf16_bits_to_double(q[c]);"),
+    "bwd_dv_drops_gate_factor": ("if (dvr) dvr[c] += pj * a * bf16_bits_to_double(dout[c]);",
+                                 "if (dvr) dvr[c] += pj * bf16_bits_to_double(dout[c]);"),
+    "bwd_dq_reads_v": ("dq[c] += scale * ds * bf16_bits_to_double(kr[c]);",
+                       "dq[c] += scale * ds * bf16_bits_to_double(vr[c]);"),
+    "bwd_local_drops_self_key": (
+        "row_grad(qr, kh, vh, er, 1.0, j_lo, i, d, pr.scale, p, o, dqr, dkh, dvh, -1);",
+        "row_grad(qr, kh, vh, er, 1.0, j_lo, i > j_lo ? i - 1 : i, d, pr.scale, p, o, dqr, dkh, dvh, -1);"),
+    "bwd_gqa_first_head_only": (
+        "for (int h = hk * G; h < (hk + 1) * G; ++h) {\n                    for (int64_t i = 0; i < len; ++i) {",
+        "for (int h = hk * G; h < hk * G + 1; ++h) {\n                    for (int64_t i = 0; i < len; ++i) {"),
 }
 
 PINS = [
@@ -66,6 +84,9 @@ PINS = [
     lambda: [dpins.test_decode_vs_dense_masks(s) for s in range(2)],
     dpins.test_decode_matches_prefill_rows,
     dpins.test_decode_closed_forms,
+    lambda: [bpins.test_backward_matches_finite_differences(c) for c in bpins.FD_CASES],
+    lambda: [bpins.test_backward_vs_sdpa_autograd(*c) for c in ((0, 16, 0.2), (3, 1, 1.0))],
+    bpins.test_backward_invariants,
 ]
 
 
