@@ -271,6 +271,82 @@ def run_decode(args, rank, world):
         print(json.dumps(line), flush=True)
 
 
+def run_train(args, rank, world):
+    """Training step (row f1): the training forward (selection, local and global branches,
+    saving the softmax statistics and both branches of the selected rows) and the backward
+    pass (dQ, dK, dV, gate gradient) at 32K tokens, Hq=32, Hkv=8, d=128, W=4096, 20% global.
+    Roofline: the backward's useful FLOPs (five matmuls per attended pair, the usual count)
+    over its own event-timed duration, against the measured bf16 peak."""
+    import token_level_dynamic_seq_b200 as logo
+    from token_level_dynamic_seq_b200 import workloads
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    w = workloads.load("c32k", seed=rank)
+    q, k, v, g = w.q.to(dev), w.k.to(dev), w.v.to(dev), w.g.to(dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1000 + rank)
+    dout = torch.randn(q.shape, generator=gen, device=dev).to(torch.bfloat16)
+    stream = torch.cuda.current_stream(dev)
+    out, ctx = logo.forward_train(q, k, v, g, w.W, w.ratio, stream=stream)
+    dq, dk, dv, dg, bws = logo.backward(q, k, v, g, out, dout, ctx, stream=stream)
+    grads = (dq, dk, dv, dg)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        logo.forward_train(q, k, v, g, w.W, w.ratio, ws=ctx["ws"], stream=stream, reuse=(out, ctx))
+        if ev is not None:
+            ev[1].record(stream)
+        logo.backward(q, k, v, g, out, dout, ctx, ws=bws, stream=stream, grads=grads)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    logo.check(ctx["ws"], stream)
+    logo.check(bws, stream)
+    tot_sel = int(ctx["cu_sel"][-1].item())
+    sel_pos = ctx["sel_idx"][:tot_sel].to(torch.int64)
+    f_loc, f_glob = logo.useful_flops(w.d, w.Hq, w.seqlens, w.W, sel_pos.tolist())
+    fwd_flops = f_loc + f_glob
+    bwd_flops = 2.5 * fwd_flops          # dS-recompute-free count: S, dP, dV, dK, dQ per pair
+    bwd_exec = 3.5 * fwd_flops           # matmuls this design issues: S and dP twice (dQ and dK/dV kernels)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    logo.check(ctx["ws"], stream)
+    logo.check(bws, stream)
+    total_ms = evs[0][0].elapsed_time(evs[-1][2]) / args.steps
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    peak_burst, peak_sust, hbm, peak_src = peaks()
+    achieved = bwd_flops / (bwd_ms * 1e-3) / 1e12
+    tokens = sum(w.seqlens)
+    line = {
+        "metric": "LoGo training step tokens/s (forward + backward, 32K tokens, 20% global)",
+        "value": tokens / (total_ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "train_c32k", "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "d": w.d, "W": w.W,
+                   "ratio": w.ratio, "selected": tot_sel, "l2": "inputs (Q 268 MB) larger than L2"},
+        "forward_ms": fwd_ms, "backward_ms": bwd_ms,
+        "backward_useful_tflops": achieved, "backward_executed_tflops": bwd_exec / (bwd_ms * 1e-3) / 1e12,
+        "roofline": {"kernel": "backward (prep, dQ selected, dQ local, dK/dV)", "bound": "tensor",
+                     "achieved": achieved, "peak": peak_burst, "unit": "TFLOP/s", "frac": achieved / peak_burst,
+                     "traffic": None, "peak_source": f"{peak_src} bf16 burst (sustained {peak_sust})"},
+        "gpu_launches": 8 * args.steps, "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -281,6 +357,9 @@ def main():
         return
     if args.workload == "decode_c32k":
         run_decode(args, rank, world)
+        return
+    if args.workload == "train_c32k":
+        run_train(args, rank, world)
         return
     assert args.warmup >= 3, "at least 3 warm-up steps"
 

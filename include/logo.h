@@ -271,6 +271,59 @@ LOGO_API logo_status logo_decode(const logo_bf16 *q, const logo_bf16 *k_cache, c
                                  int32_t *selected, void *ws, size_t ws_bytes, logo_stream_t stream);
 
 /*
+ * Training forward: logo_forward plus what the backward pass needs ("LoGo",
+ * Abstract, and "Learning When to Attend", "Empirical Validation and System
+ * Optimization": the gate is learned with the model and the kernels are
+ * claimed to speed up training).  Same arguments and results as logo_forward,
+ * and in addition (all device, caller-owned, overwritten):
+ *   sel_capacity  rows the selection list may hold (>= cu_sel[nseq]; the
+ *                 row stride of lse_sel and glob; a larger selection is an
+ *                 error the kernels report in the status word);
+ *   lse      fp32 [B*Hq][L]: per row, log2 of the local softmax's normaliser
+ *            in the scaled-score exp2 domain (m * scale * log2(e) + log2(sum));
+ *            rows of a packed tensor that lie in no sequence are not written;
+ *   lse_sel  fp32 [Hq][sel_capacity]: the same for the global softmax of each
+ *            selected row (row r of the selection list, all sequences);
+ *   glob     bf16 [Hq][sel_capacity][d]: the global branch of each selected
+ *            row before the gate;
+ *   loc_sel  bf16 [Hq][sel_capacity][d]: the local branch of each selected
+ *            row (its value before the merge).
+ */
+LOGO_API logo_status logo_forward_train(const logo_bf16 *q, const logo_bf16 *k, const logo_bf16 *v, const float *gate,
+                                        const logo_shape *shape, int window, double ratio, float scale,
+                                        logo_bf16 *out, int32_t *sel_idx, int32_t *cu_sel, int sel_capacity,
+                                        float *lse, float *lse_sel, logo_bf16 *glob, logo_bf16 *loc_sel, void *ws,
+                                        size_t ws_bytes, logo_stream_t stream);
+
+/*
+ * Backward pass: gradients of a scalar loss given dout = dL/d(out), for the
+ * forward pass logo_forward_train ran on the same q, k, v, gate, shape,
+ * window and scale.  The pages print no backward formulas; this is the chain
+ * rule through the forward definition, with the reading that out depends on
+ * gate[i] only through sigmoid(gate[i]) on selected rows (the selection is a
+ * step function and passes no gradient):
+ *   dgate[i] = sigmoid'(gate[i]) * sum_h <dout[h,i], global[h,i]> on selected
+ *              rows, 0 on every other row;
+ *   dq, dk, dv  through both softmax branches, the global one with upstream
+ *              gradient sigmoid(gate[i]) * dout[h,i]; dk and dv sum over the
+ *              query heads of a GQA group.
+ * Inputs: q, k, v, gate, out (the forward's output), dout [B, Hq, L, d] bf16;
+ * sel_idx, cu_sel, sel_capacity, lse, lse_sel, glob, loc_sel as the forward left them;
+ * max_selected bounds every sequence's count (as for logo_global_attn_sparse).
+ * Outputs (device, overwritten): dq [B, Hq, L, d], dk, dv [B, Hkv, L, d] bf16,
+ * dgate [B*L] fp32.  Rows of a packed tensor that lie in no sequence are left
+ * as they were in dq, dk and dv.  The workspace must hold
+ * logo_backward_workspace_size(shape, sel_capacity) bytes.
+ */
+LOGO_API size_t logo_backward_workspace_size(const logo_shape *shape, int sel_capacity);
+LOGO_API logo_status logo_backward(const logo_bf16 *q, const logo_bf16 *k, const logo_bf16 *v, const float *gate,
+                                   const logo_bf16 *out, const logo_bf16 *dout, const int32_t *sel_idx,
+                                   const int32_t *cu_sel, int sel_capacity, int max_selected, const float *lse,
+                                   const float *lse_sel, const logo_bf16 *glob, const logo_bf16 *loc_sel,
+                                   const logo_shape *shape, int window, float scale, logo_bf16 *dq, logo_bf16 *dk,
+                                   logo_bf16 *dv, float *dgate, void *ws, size_t ws_bytes, logo_stream_t stream);
+
+/*
  * Synchronise `stream`, then report: LOGO_ERR_CUDA if a launch or the stream
  * failed, LOGO_ERR_DEVICE_TIMEOUT if a kernel recorded a bounded wait that ran
  * out, LOGO_ERR_INVALID_ARG if a kernel recorded an argument it could not

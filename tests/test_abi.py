@@ -32,7 +32,7 @@ def declared_symbols():
 def test_library_exports_every_declared_symbol():
     lib = logo.load_library()
     names = declared_symbols()
-    assert len(names) == 16, names
+    assert len(names) == 19, names
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(logo.EXPORTED)
@@ -131,3 +131,34 @@ def test_select_and_forward_reject():
     # selftest: bad limits
     assert lib.logo_selftest_timeout(FAKE, 256, 0, None) == 1
     assert lib.logo_selftest_timeout(None, 256, 10, None) == 3
+
+
+@no_gpu_only
+def test_training_entry_points_reject():
+    lib = logo.load_library()
+    sh = shape()
+    by = ctypes.byref(sh)
+    assert lib.logo_backward_workspace_size(by, 64) > 256
+    assert lib.logo_backward_workspace_size(by, -1) == 0
+    assert lib.logo_backward_workspace_size(ctypes.byref(shape(d=96)), 64) == 0
+    ft = lambda **kw: lib.logo_forward_train(
+        FAKE, FAKE, FAKE, FAKE, kw.get("by", by), kw.get("window", 8), kw.get("ratio", 0.2), 0.0, FAKE2, FAKE, FAKE,
+        kw.get("cap", 64), kw.get("lse", FAKE), FAKE, FAKE, FAKE, FAKE, 256, None)
+    assert ft(window=0) == 1
+    assert ft(ratio=1.5) == 1
+    assert ft(cap=-1) == 1
+    assert ft(cap=10) == 1          # below one sequence's count (52 of 256)
+    assert ft(lse=None) == 1
+    assert ft(by=ctypes.byref(shape(d=96))) == 2
+    need = lib.logo_backward_workspace_size(by, 64)
+    bw = lambda **kw: lib.logo_backward(
+        FAKE, FAKE, FAKE, FAKE, FAKE, kw.get("dout", FAKE), FAKE, FAKE, kw.get("cap", 64), kw.get("max_sel", 52),
+        FAKE, FAKE, FAKE, FAKE, by, kw.get("window", 8), 0.0, FAKE2, FAKE2, FAKE2, FAKE2, FAKE,
+        kw.get("ws_bytes", need),
+        None)
+    assert bw(window=0) == 1
+    assert bw(max_sel=65) == 1      # above the capacity
+    assert bw(max_sel=-1) == 1
+    assert bw(ws_bytes=need - 1) == 3
+    assert bw(dout=None) == 1
+    assert lib.logo_last_error().decode() != ""

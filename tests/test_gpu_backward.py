@@ -1,0 +1,124 @@
+"""Backward pass on the GPU against the fp64 oracle's backward.
+
+The training forward must give the same output as the plain forward (it
+only saves statistics besides).  Gradients are compared element by element
+with the oracle on small problems (several tiles and ragged tails, GQA,
+packed sequences, W = 1, ratio 0 and 1), and at the 32K headline size on
+sampled rows the oracle computes one by one plus two sums that hold at any
+size (the key gradients of a key/value head sum to zero; the value gradients
+sum to the upstream gradients they received).
+
+Tolerance: relative L2 error <= 5e-3 (the forward's budget) and max-abs
+error <= 1e-2 of the largest reference magnitude, per gradient.  The kernels
+round P and dS to bf16 for the tensor cores, read the bf16 branch outputs for
+D = <dout, o> and write bf16 gradients; each rounding contributes about
+2^-9 / sqrt(3) ~ 1.1e-3 relative, and they add in quadrature to ~2.5e-3.
+"""
+import pytest
+import torch
+
+import oracle
+import token_level_dynamic_seq_b200 as logo
+from token_level_dynamic_seq_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 5e-3
+MAX_ABS_FRAC = 1e-2
+
+
+def close(got, ref, what):
+    got = got.double().cpu()
+    ref = ref.double()
+    assert torch.isfinite(got).all(), f"{what}: non-finite values"
+    scale = ref.abs().max().item()
+    err = (got - ref).abs().max().item()
+    rel = ((got - ref).norm() / ref.norm().clamp_min(1e-30)).item()
+    print(f"{what}: max-abs {err:.3e} (ref max {scale:.3e}) rel-L2 {rel:.3e}")
+    assert rel <= REL_L2 and err <= MAX_ABS_FRAC * max(scale, 1e-30), \
+        f"{what}: max-abs {err:.3e} of {scale:.3e}, rel-L2 {rel:.3e}"
+
+
+def gpu_run(w, e):
+    cu = None if w.cu_seqlens is None else w.cu_seqlens.cuda()
+    ml = None if w.cu_seqlens is None else max(w.seqlens)
+    q, k, v, g = w.q.cuda(), w.k.cuda(), w.v.cuda(), w.g.cuda()
+    out, ctx = logo.forward_train(q, k, v, g, w.W, w.ratio, cu_seqlens=cu, max_seqlen=ml)
+    dq, dk, dv, dg, ws = logo.backward(q, k, v, g, out, e.cuda(), ctx)
+    logo.check(ctx["ws"])
+    logo.check(ws)
+    plain, _, _ = logo.forward(q, k, v, g, w.W, w.ratio, cu_seqlens=cu, max_seqlen=ml)
+    torch.cuda.synchronize()
+    assert torch.equal(out, plain), "training forward changed the output"
+    return dq, dk, dv, dg
+
+
+CASES = {
+    # name: (B, Hq, Hkv, L, d, W, ratio, seqlens)
+    "mha_d128": (1, 2, 2, 300, 128, 64, 0.25, None),
+    "gqa_d128_b2": (2, 4, 2, 513, 128, 100, 0.3, None),
+    "gqa4_d64": (1, 8, 2, 700, 64, 256, 0.2, None),
+    "w1": (1, 2, 1, 260, 128, 1, 0.5, None),
+    "ratio0": (1, 2, 1, 390, 128, 50, 0.0, None),
+    "ratio1_full_window": (1, 2, 2, 200, 128, 4096, 1.0, None),
+    "group3": (1, 3, 1, 333, 128, 77, 0.4, None),
+    "varlen": (1, 4, 2, 0, 128, 128, 0.25, [300, 1, 0, 257, 129, 640]),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_backward_small_full(name):
+    B, Hq, Hkv, L, d, W, ratio, lens = CASES[name]
+    w = workloads.make(B, Hq, Hkv, L, d, W, ratio, seed=len(name), qkv_scale=1.0, seqlens=lens)
+    gen = torch.Generator().manual_seed(17 + len(name))
+    e = torch.randn(w.q.shape, generator=gen).bfloat16()
+    dq, dk, dv, dg = gpu_run(w, e)
+    ref = oracle.backward(w.q, w.k, w.v, w.g, e, w.W, w.ratio, cu_seqlens=w.cu_seqlens)
+    if w.cu_seqlens is not None:
+        T = int(w.cu_seqlens[-1])
+        sl = (slice(None), slice(None), slice(0, T))
+        dq, dk, dv = dq[sl], dk[sl], dv[sl]
+        ref = {kk: (vv[sl] if kk in ("dq", "dk", "dv") else vv) for kk, vv in ref.items()}
+        dg = dg[:, :T]
+        ref["dg"] = ref["dg"][:, :T]
+    close(dq, ref["dq"], f"{name} dq")
+    close(dk, ref["dk"], f"{name} dk")
+    close(dv, ref["dv"], f"{name} dv")
+    if ratio > 0:
+        close(dg, ref["dg"], f"{name} dgate")
+        assert (dg.cpu()[ref["dg"] == 0] == 0).all(), "gate gradient off the selection"
+    else:
+        assert (dg == 0).all()
+
+
+def test_backward_headline_sampled():
+    """32K tokens, Hq=32, Hkv=8, d=128, W=4096, 20% global: sampled rows and sums."""
+    w = workloads.load("c32k")
+    gen = torch.Generator().manual_seed(5)
+    e = torch.randn(w.q.shape, generator=gen).bfloat16()
+    dq, dk, dv, dg = gpu_run(w, e)
+    L = w.L
+    flags = oracle.selection_flags(w.g, w.ratio)
+    sel = flags[0].nonzero().flatten().tolist()
+    qrows = [(0, 0, 0), (0, 31, L - 1), (0, 5, 4095), (0, 12, 4096), (0, 20, sel[0]), (0, 7, sel[len(sel) // 2]),
+             (0, 30, sel[-1]), (0, 1, 16385)]
+    krows = [(0, 0, L - 1), (0, 7, L - 130), (0, 3, L - 129), (0, 5, L - 200)]
+    ref = oracle.backward_rows(w.q, w.k, w.v, w.g, e, w.W, w.ratio, qrows=qrows, krows=krows, flags=flags)
+    got_q = torch.stack([dq[0, h, i] for _, h, i in qrows])
+    close(got_q, ref["dq"], "c32k dq rows")
+    got_g = torch.stack([dg[0, i] for _, _, i in qrows])
+    sel_rows = [t for t, (_, _, i) in enumerate(qrows) if flags[0, i]]
+    close(got_g[sel_rows], ref["dg"][sel_rows], "c32k dgate rows")
+    close(torch.stack([dk[0, h, j] for _, h, j in krows]), ref["dk"], "c32k dk rows")
+    close(torch.stack([dv[0, h, j] for _, h, j in krows]), ref["dv"], "c32k dv rows")
+    # sums over all keys of a head (fp64 on the host)
+    G = w.Hq // w.Hkv
+    sg = torch.sigmoid(w.g[0].double())
+    weight = 1.0 + torch.where(flags[0].bool(), sg, torch.zeros_like(sg))
+    ed = e[0].double() * weight.view(1, -1, 1)
+    want_v = ed.view(w.Hkv, G, L, w.d).sum((1, 2))
+    got_v = dv[0].double().cpu().sum(1)
+    close(got_v, want_v, "c32k sum of dv per head")
+    dk_abs = dk[0].double().cpu().abs().sum(1)
+    dk_sum = dk[0].double().cpu().sum(1)
+    assert (dk_sum.abs() <= 2e-2 * dk_abs).all(), "key gradients of a head must sum to ~0"

@@ -35,7 +35,8 @@ EXPORTED = ("logo_num_selected", "logo_workspace_size", "logo_workspace_init", "
             "logo_local_attn", "logo_global_attn_sparse", "logo_forward", "logo_check",
             "logo_selftest_timeout", "logo_status_string", "logo_last_error",
             "logo_global_attn_sparse_noalloc", "logo_select_threshold", "logo_threshold_update",
-            "logo_decode_workspace_size", "logo_decode")
+            "logo_decode_workspace_size", "logo_decode", "logo_forward_train", "logo_backward_workspace_size",
+            "logo_backward")
 
 
 class LogoError(RuntimeError):
@@ -85,6 +86,11 @@ def load_library(path: str | None = None):
             "logo_threshold_update": ([vp, sp, dbl, flt, vp, vp, vp, sz, vp], i32),
             "logo_decode_workspace_size": ([sp], sz),
             "logo_decode": ([vp, vp, vp, vp, vp, vp, sp, i32, flt, vp, vp, vp, sz, vp], i32),
+            "logo_forward_train": ([vp, vp, vp, vp, sp, i32, dbl, flt, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp],
+                                   i32),
+            "logo_backward_workspace_size": ([sp, i32], sz),
+            "logo_backward": ([vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sp, i32, flt, vp, vp, vp,
+                               vp, vp, sz, vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -273,6 +279,77 @@ def forward(q, k, v, gate, window: int, ratio: float, ws: torch.Tensor | None = 
                                        float(ratio), float(scale), _ptr(out), _ptr(sel_idx), _ptr(cu_sel),
                                        _ptr(ws), ws.numel(), _stream(stream)))
     return out, sel_idx, cu_sel
+
+
+def forward_train(q, k, v, gate, window: int, ratio: float, ws: torch.Tensor | None = None, scale: float = 0.0,
+                  cu_seqlens=None, max_seqlen=None, stream=None, reuse=None):
+    """Forward pass that also saves what :func:`backward` needs.
+
+    Returns (out, ctx): ``ctx`` holds the selection (sel_idx, cu_sel, its
+    capacity and the largest per-sequence count) and the saved statistics
+    (lse [B*Hq*L], lse_sel [Hq, cap], glob and loc_sel [Hq, cap, d]: the two
+    branches of the selected rows).  ``reuse`` = (out, ctx) of an earlier call
+    with the same shapes: its buffers are written again instead of new ones."""
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    shape = make_shape(q, k, cu_seqlens, max_seqlen)
+    if ws is None:
+        ws = workspace(shape, ratio, q.device, stream)
+    dev = q.device
+    nseq = shape.nseq if cu_seqlens is not None else shape.B
+    cap = max(1, selection_capacity(shape, ratio))
+    max_sel = num_selected(ratio, shape.max_seqlen)
+    if reuse is not None:
+        out, old = reuse
+        sel_idx, cu_sel, lse, lse_sel, glob, loc_sel = (old[n] for n in ("sel_idx", "cu_sel", "lse", "lse_sel",
+                                                                           "glob", "loc_sel"))
+        cap = old["cap"]
+    else:
+        out = torch.empty_like(q)
+        sel_idx = torch.empty(cap, dtype=torch.int32, device=dev)
+        cu_sel = torch.empty(nseq + 1, dtype=torch.int32, device=dev)
+        lse = torch.empty(q.shape[0] * q.shape[1] * q.shape[2], dtype=torch.float32, device=dev)
+        lse_sel = torch.empty(q.shape[1], cap, dtype=torch.float32, device=dev)
+        glob = torch.empty(q.shape[1], cap, q.shape[3], dtype=torch.bfloat16, device=dev)
+        loc_sel = torch.empty_like(glob)
+    _raise(load_library().logo_forward_train(_ptr(q), _ptr(k), _ptr(v), _ptr(gate), ctypes.byref(shape), int(window),
+                                             float(ratio), float(scale), _ptr(out), _ptr(sel_idx), _ptr(cu_sel), cap,
+                                             _ptr(lse), _ptr(lse_sel), _ptr(glob), _ptr(loc_sel), _ptr(ws),
+                                             ws.numel(),
+                                             _stream(stream)))
+    ctx = {"sel_idx": sel_idx, "cu_sel": cu_sel, "cap": cap, "max_selected": max_sel, "lse": lse,
+           "lse_sel": lse_sel, "glob": glob, "loc_sel": loc_sel, "window": int(window), "scale": float(scale),
+           "shape": shape, "ws": ws}
+    return out, ctx
+
+
+def backward_workspace(shape: Shape, cap: int, device) -> torch.Tensor:
+    n = load_library().logo_backward_workspace_size(ctypes.byref(shape), int(cap))
+    if n == 0:
+        _raise(1)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return ws
+
+
+def backward(q, k, v, gate, out, dout, ctx, ws: torch.Tensor | None = None, stream=None, grads=None):
+    """Gradients (dq, dk, dv, dgate) of a loss with dL/d(out) = dout, for a forward
+    pass made by :func:`forward_train` (its ``ctx``).  ``grads`` may hold
+    preallocated outputs (dq, dk, dv, dgate)."""
+    q, k, v, out, dout = _bits(q), _bits(k), _bits(v), _bits(out), _bits(dout)
+    shape = ctx["shape"]
+    if ws is None:
+        ws = backward_workspace(shape, ctx["cap"], q.device)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+                 torch.empty(gate.shape, dtype=torch.float32, device=q.device))
+    dq, dk, dv, dg = grads
+    _raise(load_library().logo_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(out), _ptr(dout),
+                                        _ptr(ctx["sel_idx"]), _ptr(ctx["cu_sel"]), ctx["cap"], ctx["max_selected"],
+                                        _ptr(ctx["lse"]), _ptr(ctx["lse_sel"]), _ptr(ctx["glob"]),
+                                        _ptr(ctx["loc_sel"]), ctypes.byref(shape), ctx["window"], ctx["scale"],
+                                        _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(ws), ws.numel(),
+                                        _stream(stream)))
+    return dq, dk, dv, dg, ws
 
 
 def selftest_timeout(ws: torch.Tensor, limit_us: int = 1000, stream=None):

@@ -165,12 +165,22 @@ void base_params(AttnParams& p, const Geo& g, const void* q, const void* k, cons
     (void)v;
 }
 
+// Statistics the training forward saves for the backward pass (all optional).
+struct SavedStats {
+    float* lse = nullptr;      // [B*Hq][L]
+    float* lse_sel = nullptr;  // [Hq][sel_stride]
+    uint16_t* glob = nullptr;  // [Hq][sel_stride][d]
+    uint16_t* loc_sel = nullptr;  // [Hq][sel_stride][d]
+    int sel_stride = 0;
+};
+
 logo_status launch_local(const Geo& g, const void* q, const void* k, const void* v, int window, float scale_log2,
-                         void* out, void* ws, cudaStream_t stream)
+                         void* out, void* ws, cudaStream_t stream, const SavedStats* saved = nullptr)
 {
     if (g.L == 0 || g.max_len == 0) return LOGO_OK;
     AttnParams p;
     base_params(p, g, q, k, v, out, scale_log2, ws);
+    if (saved) p.lse = saved->lse;
     p.window = window < g.max_len ? window : (g.max_len > 0 ? g.max_len : 1);
     logo_status st;
     if ((st = make_map(&p.tm_q, q, g.d, g.L, g.B * g.Hq)) != LOGO_OK) return st;
@@ -183,11 +193,17 @@ logo_status launch_local(const Geo& g, const void* q, const void* k, const void*
 
 logo_status launch_global(const Geo& g, const void* q, const void* k, const void* v, const float* gate,
                           const int32_t* sel_idx, const int32_t* cu_sel, int max_selected, float scale_log2,
-                          int merge, void* out, void* ws, cudaStream_t stream)
+                          int merge, void* out, void* ws, cudaStream_t stream, const SavedStats* saved = nullptr)
 {
     if (g.L == 0 || g.max_len == 0 || max_selected == 0) return LOGO_OK;
     AttnParams p;
     base_params(p, g, q, k, v, out, scale_log2, ws);
+    if (saved) {
+        p.lse = saved->lse_sel;
+        p.glob = saved->glob;
+        p.loc_sel = saved->loc_sel;
+        p.sel_stride = saved->sel_stride;
+    }
     p.gate = gate;
     p.sel_idx = sel_idx;
     p.cu_sel = cu_sel;
@@ -211,6 +227,39 @@ void logo::set_last_error(const char* fmt, ...)
     vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
     va_end(ap);
 }
+
+namespace {
+
+// Backward workspace: header | D of local rows | D of selected rows | row -> list slot |
+// Q of selected rows | sigmoid(g) dout of selected rows | fp32 dQ of selected rows.
+struct BwdWs {
+    size_t dl, ds_sel, slot, q_sel, do_sel, dq_sel, total;
+};
+
+size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+
+BwdWs bwd_layout(const Geo& g, int cap)
+{
+    BwdWs w;
+    size_t off = kWsHeaderBytes;
+    const size_t rows = (size_t)g.B * g.Hq * g.L, sel = (size_t)g.Hq * (size_t)cap;
+    w.dl = off;
+    off += round256(rows * 4);
+    w.ds_sel = off;
+    off += round256(sel * 4);
+    w.slot = off;
+    off += round256((size_t)g.B * g.L * 4);
+    w.q_sel = off;
+    off += round256(sel * g.d * 2);
+    w.do_sel = off;
+    off += round256(sel * g.d * 2);
+    w.dq_sel = off;
+    off += round256(sel * g.d * 4);
+    w.total = off;
+    return w;
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -319,6 +368,165 @@ logo_status logo_forward(const logo_bf16* q, const logo_bf16* k, const logo_bf16
     if ((st = logo_select(gate, shape, ratio, sel_idx, cu_sel, ws, ws_bytes, stream)) != LOGO_OK) return st;
     if ((st = launch_local(g, q, k, v, window, sl2, out, ws, s)) != LOGO_OK) return st;
     return launch_global(g, q, k, v, gate, sel_idx, cu_sel, max_sel, sl2, 1, out, ws, s);
+}
+
+logo_status logo_forward_train(const logo_bf16* q, const logo_bf16* k, const logo_bf16* v, const float* gate,
+                               const logo_shape* shape, int window, double ratio, float scale, logo_bf16* out,
+                               int32_t* sel_idx, int32_t* cu_sel, int sel_capacity, float* lse, float* lse_sel,
+                               logo_bf16* glob, logo_bf16* loc_sel, void* ws, size_t ws_bytes, logo_stream_t stream)
+{
+    Geo g;
+    logo_status st;
+    float sl2;
+    if ((st = check_shape(shape, g)) != LOGO_OK) return st;
+    if ((st = check_ratio(ratio)) != LOGO_OK) return st;
+    if (window < 1) return fail(LOGO_ERR_INVALID_ARG, "window=%d must be >= 1", window);
+    if ((st = resolve_scale(scale, g.d, sl2)) != LOGO_OK) return st;
+    if ((st = check_ws(ws, ws_bytes)) != LOGO_OK) return st;
+    if ((st = check_ptr(cu_sel, "cu_sel")) != LOGO_OK) return st;
+    const int max_sel = (int)logo::budget_count(ratio, g.max_len);
+    if (sel_capacity < 0) return fail(LOGO_ERR_INVALID_ARG, "sel_capacity=%d must be >= 0", sel_capacity);
+    if (max_sel > 0 && sel_capacity < max_sel)
+        return fail(LOGO_ERR_INVALID_ARG, "sel_capacity=%d is below one sequence's count %d", sel_capacity, max_sel);
+    if (g.L > 0) {
+        if ((st = check_ptr(q, "q")) != LOGO_OK || (st = check_ptr(k, "k")) != LOGO_OK ||
+            (st = check_ptr(v, "v")) != LOGO_OK || (st = check_ptr(out, "out")) != LOGO_OK ||
+            (st = check_ptr(gate, "gate")) != LOGO_OK || (st = check_ptr(lse, "lse")) != LOGO_OK)
+            return st;
+        if (max_sel > 0 && ((st = check_ptr(sel_idx, "sel_idx")) != LOGO_OK ||
+                            (st = check_ptr(lse_sel, "lse_sel")) != LOGO_OK || (st = check_ptr(glob, "glob")) != LOGO_OK ||
+                            (st = check_ptr(loc_sel, "loc_sel")) != LOGO_OK))
+            return st;
+    }
+    SavedStats saved;
+    saved.lse = lse;
+    saved.lse_sel = lse_sel;
+    saved.glob = reinterpret_cast<uint16_t*>(glob);
+    saved.loc_sel = reinterpret_cast<uint16_t*>(loc_sel);
+    saved.sel_stride = sel_capacity;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = logo_select(gate, shape, ratio, sel_idx, cu_sel, ws, ws_bytes, stream)) != LOGO_OK) return st;
+    if ((st = launch_local(g, q, k, v, window, sl2, out, ws, s, &saved)) != LOGO_OK) return st;
+    return launch_global(g, q, k, v, gate, sel_idx, cu_sel, max_sel, sl2, 1, out, ws, s, &saved);
+}
+
+size_t logo_backward_workspace_size(const logo_shape* shape, int sel_capacity)
+{
+    Geo g;
+    if (check_shape(shape, g) != LOGO_OK || sel_capacity < 0) return 0;
+    return bwd_layout(g, sel_capacity).total;
+}
+
+logo_status logo_backward(const logo_bf16* q, const logo_bf16* k, const logo_bf16* v, const float* gate,
+                          const logo_bf16* out, const logo_bf16* dout, const int32_t* sel_idx, const int32_t* cu_sel,
+                          int sel_capacity, int max_selected, const float* lse, const float* lse_sel,
+                          const logo_bf16* glob, const logo_bf16* loc_sel, const logo_shape* shape, int window,
+                          float scale, logo_bf16* dq,
+                          logo_bf16* dk, logo_bf16* dv, float* dgate, void* ws, size_t ws_bytes,
+                          logo_stream_t stream)
+{
+    Geo g;
+    logo_status st;
+    float sl2;
+    if ((st = check_shape(shape, g)) != LOGO_OK) return st;
+    if (window < 1) return fail(LOGO_ERR_INVALID_ARG, "window=%d must be >= 1", window);
+    if ((st = resolve_scale(scale, g.d, sl2)) != LOGO_OK) return st;
+    if (sel_capacity < 0) return fail(LOGO_ERR_INVALID_ARG, "sel_capacity=%d must be >= 0", sel_capacity);
+    if (max_selected < 0 || max_selected > g.max_len || max_selected > sel_capacity)
+        return fail(LOGO_ERR_INVALID_ARG, "max_selected=%d outside [0, min(%d, sel_capacity=%d)]", max_selected,
+                    g.max_len, sel_capacity);
+    if ((st = check_ws(ws, ws_bytes)) != LOGO_OK) return st;
+    const BwdWs lay = bwd_layout(g, sel_capacity);
+    if (ws_bytes < lay.total)
+        return fail(LOGO_ERR_WORKSPACE, "backward workspace of %zu bytes, need %zu", ws_bytes, lay.total);
+    if (g.L == 0 || g.max_len == 0) return LOGO_OK;
+    if ((st = check_ptr(q, "q")) != LOGO_OK || (st = check_ptr(k, "k")) != LOGO_OK ||
+        (st = check_ptr(v, "v")) != LOGO_OK || (st = check_ptr(gate, "gate")) != LOGO_OK ||
+        (st = check_ptr(out, "out")) != LOGO_OK || (st = check_ptr(dout, "dout")) != LOGO_OK ||
+        (st = check_ptr(lse, "lse")) != LOGO_OK || (st = check_ptr(cu_sel, "cu_sel")) != LOGO_OK ||
+        (st = check_ptr(dq, "dq")) != LOGO_OK || (st = check_ptr(dk, "dk")) != LOGO_OK ||
+        (st = check_ptr(dv, "dv")) != LOGO_OK || (st = check_ptr(dgate, "dgate")) != LOGO_OK)
+        return st;
+    const bool any_sel = max_selected > 0;
+    if (any_sel && ((st = check_ptr(sel_idx, "sel_idx")) != LOGO_OK || (st = check_ptr(lse_sel, "lse_sel")) != LOGO_OK ||
+                    (st = check_ptr(glob, "glob")) != LOGO_OK || (st = check_ptr(loc_sel, "loc_sel")) != LOGO_OK))
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* wb = static_cast<uint8_t*>(ws);
+    float* dl = reinterpret_cast<float*>(wb + lay.dl);
+    float* ds_sel = reinterpret_cast<float*>(wb + lay.ds_sel);
+    int32_t* slot = reinterpret_cast<int32_t*>(wb + lay.slot);
+    uint16_t* q_sel = reinterpret_cast<uint16_t*>(wb + lay.q_sel);
+    uint16_t* do_sel = reinterpret_cast<uint16_t*>(wb + lay.do_sel);
+    float* dq_sel = reinterpret_cast<float*>(wb + lay.dq_sel);
+
+    logo::PrepParams pp;
+    memset(&pp, 0, sizeof pp);
+    pp.q = static_cast<const uint16_t*>(q);
+    pp.out = static_cast<const uint16_t*>(out);
+    pp.dout = static_cast<const uint16_t*>(dout);
+    pp.glob = static_cast<const uint16_t*>(glob);
+    pp.loc_sel = static_cast<const uint16_t*>(loc_sel);
+    pp.gate = gate;
+    pp.cu_seqlens = g.cu;
+    pp.sel_idx = sel_idx;
+    pp.cu_sel = any_sel ? cu_sel : nullptr;
+    pp.dl = dl;
+    pp.ds_sel = ds_sel;
+    pp.dgate = dgate;
+    pp.slot = slot;
+    pp.q_sel = q_sel;
+    pp.do_sel = do_sel;
+    pp.status = static_cast<uint32_t*>(ws);
+    pp.B = g.B;
+    pp.Hq = g.Hq;
+    pp.L = g.L;
+    pp.nseq = g.nseq;
+    pp.sel_stride = any_sel ? sel_capacity : 0;
+    cudaError_t e = logo::launch_bwd_prep(pp, g.d, s);
+    if (e != cudaSuccess) return cuda_fail(e, "backward prep launch");
+
+    logo::BwdParams p;
+    memset(&p, 0, sizeof p);
+    if ((st = make_map(&p.tm_q, q, g.d, g.L, g.B * g.Hq)) != LOGO_OK) return st;
+    if ((st = make_map(&p.tm_do, dout, g.d, g.L, g.B * g.Hq)) != LOGO_OK) return st;
+    if ((st = make_map(&p.tm_k, k, g.d, g.L, g.B * g.Hkv)) != LOGO_OK) return st;
+    if ((st = make_map(&p.tm_v, v, g.d, g.L, g.B * g.Hkv)) != LOGO_OK) return st;
+    if (any_sel) {
+        if ((st = make_map(&p.tm_qs, q_sel, g.d, sel_capacity, g.Hq)) != LOGO_OK) return st;
+        if ((st = make_map(&p.tm_dos, do_sel, g.d, sel_capacity, g.Hq)) != LOGO_OK) return st;
+    }
+    p.lse = lse;
+    p.dl = dl;
+    p.lse_s = lse_sel;
+    p.ds_sel = ds_sel;
+    p.cu_seqlens = g.cu;
+    p.sel_idx = sel_idx;
+    p.cu_sel = cu_sel;
+    p.slot = slot;
+    p.dq_sel = any_sel ? dq_sel : nullptr;
+    p.dq = reinterpret_cast<uint16_t*>(dq);
+    p.dk = reinterpret_cast<uint16_t*>(dk);
+    p.dv = reinterpret_cast<uint16_t*>(dv);
+    p.status = static_cast<uint32_t*>(ws);
+    p.Hq = g.Hq;
+    p.Hkv = g.Hkv;
+    p.G = g.G;
+    p.L = g.L;
+    p.nseq = g.nseq;
+    p.window = window < g.max_len ? window : g.max_len;
+    p.max_selected = max_selected;
+    p.sel_stride = sel_capacity;
+    p.scale_log2 = sl2;
+    p.scale = scale > 0.f ? scale : (float)(1.0 / std::sqrt((double)g.d));
+    p.timeout_ns = 1000000000ull;
+    if (any_sel && (e = logo::launch_bwd_dq(logo::kModeGlobal, g.d, p, g.max_len, s)) != cudaSuccess)
+        return cuda_fail(e, "backward dQ (selected rows) launch");
+    if ((e = logo::launch_bwd_dq(logo::kModeLocal, g.d, p, g.max_len, s)) != cudaSuccess)
+        return cuda_fail(e, "backward dQ launch");
+    if ((e = logo::launch_bwd_dkdv(g.d, p, g.max_len, s)) != cudaSuccess)
+        return cuda_fail(e, "backward dK/dV launch");
+    return LOGO_OK;
 }
 
 logo_status logo_select_threshold(const float* gate, const logo_shape* shape, const float* tau, int max_selected,

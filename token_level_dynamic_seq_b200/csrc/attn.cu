@@ -66,9 +66,6 @@ static_assert(kPParts == 2, "P is published in two parts, one per half-row warpg
 // Every kPolyEvery-th exponential of a row uses exp2_poly (FMA pipe) instead
 // of the MUFU unit; 0 keeps them all on MUFU.
 constexpr int kPolyEvery = LOGO_POLY_EVERY;
-#ifndef LOGO_EXP_BATCH
-#define LOGO_EXP_BATCH 0
-#endif
 __device__ __forceinline__ constexpr bool use_poly(int col)
 {
     return kPolyEvery > 0 && (col % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
@@ -160,6 +157,10 @@ __device__ Work make_work(const AttnParams& p)
             return w;
         }
         if (k <= 0) return w;
+        if (p.lse && p.cu_sel[seq + 1] > p.sel_stride) {
+            if (threadIdx.x == 0) atomicOr(p.status, kStatusBadArgument);
+            return w;
+        }
         const int nch = ceil_div(k, kTileM);
         if (p.pair_heads) {
             const int c = nch - 1 - (int)blockIdx.y;
@@ -483,19 +484,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t pk[16];
-#if LOGO_EXP_BATCH
-                // all 32 arguments, then all 32 exponentials, then packing and sums
-                float xx[32];
-                #pragma unroll
-                for (int e = 0; e < 32; ++e) xx[e] = fmaf(__uint_as_float(sr[c][e]), sl2, -mref);
-                #pragma unroll
-                for (int e = 0; e < 32; ++e) xx[e] = use_poly(64 * half + c * 32 + e) ? exp2_poly(xx[e]) : fast_exp2(xx[e]);
-                #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    ls[(e >> 1) & 3] += xx[e] + xx[e + 1];
-                    pk[e / 2] = pack_bf16x2(xx[e], xx[e + 1]);
-                }
-#else
                 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                     const int col = 64 * half + c * 32 + e;
@@ -507,7 +495,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     ls[(e >> 1) & 3] += p0 + p1;
                     pk[e / 2] = pack_bf16x2(p0, p1);
                 }
-#endif
                 tmem_st16(tP + c * 16, pk);
             }
             l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
@@ -541,6 +528,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             const float l_row = l_run + xch[(half ^ 1) * 128 + r];
             const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
             uint16_t* orow = p.out + ((size_t)zq * p.L + w.s0 + pos) * D + (D / 2) * half;
+            // Saved for the backward pass: the row's log-sum-exp (exp2 domain) and,
+            // for selected rows, the global branch before the gate.
+            const size_t srow = MODE == kModeGlobal ? (size_t)head * p.sel_stride + w.sel_base + my_row0 + r : 0;
+            if (p.lse && row_valid && half == 0) {
+                const float lse2 = l_row > 0.f ? m_run * sl2 + log2f(l_row) : INFINITY;
+                if (MODE == kModeLocal) p.lse[(size_t)zq * p.L + w.s0 + pos] = lse2;
+                else p.lse[srow] = lse2;
+            }
+            uint16_t* grow = (MODE == kModeGlobal && p.glob) ? p.glob + srow * D + (D / 2) * half : nullptr;
+            uint16_t* lrow = (MODE == kModeGlobal && p.loc_sel) ? p.loc_sel + srow * D + (D / 2) * half : nullptr;
             float gsig = 0.f;
             if (MODE == kModeGlobal && p.merge && row_valid) {
                 const float g = p.gate[(size_t)w.b * p.L + w.s0 + pos];
@@ -557,10 +554,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 #pragma unroll
                 for (int e = 0; e < 32; ++e) vals[e] = __uint_as_float(orr[e]) * inv_l;
                 int4* dst = reinterpret_cast<int4*>(orow + c * 32);
+                if (MODE == kModeGlobal && grow) {
+                    int4* gdst = reinterpret_cast<int4*>(grow + c * 32);
+                    #pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        int4 o;
+                        o.x = (int)pack_bf16x2(vals[u * 8 + 0], vals[u * 8 + 1]);
+                        o.y = (int)pack_bf16x2(vals[u * 8 + 2], vals[u * 8 + 3]);
+                        o.z = (int)pack_bf16x2(vals[u * 8 + 4], vals[u * 8 + 5]);
+                        o.w = (int)pack_bf16x2(vals[u * 8 + 6], vals[u * 8 + 7]);
+                        gdst[u] = o;
+                    }
+                }
                 if (MODE == kModeGlobal && p.merge) {
                     #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         int4 loc = dst[u];
+                        if (lrow) reinterpret_cast<int4*>(lrow + c * 32)[u] = loc;
                         const uint32_t lw[4] = {(uint32_t)loc.x, (uint32_t)loc.y, (uint32_t)loc.z, (uint32_t)loc.w};
                         #pragma unroll
                         for (int t = 0; t < 4; ++t) {

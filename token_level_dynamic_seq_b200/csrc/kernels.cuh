@@ -63,6 +63,15 @@ struct alignas(64) AttnParams {
     int merge;
     float scale_log2;  // softmax scale * log2(e)
     unsigned long long timeout_ns;
+    // Statistics for the backward pass (training forward); nullptr: not saved.
+    //   local mode:  lse [B*Hq][L]        log-sum-exp per row, log2 units of the scaled score
+    //   global mode: lse [Hq][sel_stride] per selected row, glob [Hq][sel_stride][d] the global
+    //                branch (bf16, before the gate), loc_sel [Hq][sel_stride][d] the local branch
+    //                of the selected rows (bf16, as the local kernel wrote it), rows indexed like sel_idx
+    float* lse;
+    uint16_t* glob;
+    uint16_t* loc_sel;
+    int sel_stride;
 };
 
 cudaError_t launch_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, double ratio,
@@ -93,6 +102,41 @@ size_t decode_partials_bytes(int B, int Hkv, int G, int Lmax, int d);
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
 
 cudaError_t launch_attn(int mode, int d, const AttnParams& p, int max_seqlen, cudaStream_t stream);
+
+// Backward pass (bwd.cu).
+struct PrepParams {
+    const uint16_t *q, *out, *dout;         // dense [B*Hq][L][d]
+    const uint16_t *glob, *loc_sel;         // [Hq][sel_stride][d]: the two branches of selected rows
+    const float* gate;                      // [B*L]
+    const int32_t *cu_seqlens, *sel_idx, *cu_sel;
+    float* dl;                              // D of the local rows [B*Hq][L]
+    float* ds_sel;                          // D of the global rows [Hq][sel_stride]
+    float* dgate;                           // [B*L]
+    int32_t* slot;                          // [B*L]: row of the selection list, or -1
+    uint16_t *q_sel, *do_sel;               // [Hq][sel_stride][d]: Q and sigmoid(g) dout of selected rows
+    uint32_t* status;
+    int B, Hq, L, nseq, sel_stride;
+};
+
+struct alignas(64) BwdParams {
+    CUtensorMap tm_q, tm_do;    // dense [B*Hq][L][d]
+    CUtensorMap tm_qs, tm_dos;  // selected rows [Hq][sel_stride][d]
+    CUtensorMap tm_k, tm_v;     // [B*Hkv][L][d]
+    const float *lse, *dl;      // [B*Hq][L]
+    const float *lse_s, *ds_sel;  // [Hq][sel_stride]
+    const int32_t *cu_seqlens, *sel_idx, *cu_sel, *slot;
+    float* dq_sel;              // [Hq][sel_stride][d] fp32: global share of dQ
+    uint16_t *dq, *dk, *dv;
+    uint32_t* status;
+    int Hq, Hkv, G, L, nseq, window, max_selected, sel_stride;
+    float scale, scale_log2;
+    unsigned long long timeout_ns;
+};
+
+cudaError_t launch_bwd_prep(const PrepParams& p, int d, cudaStream_t stream);
+cudaError_t launch_bwd_dq(int mode, int d, const BwdParams& p, int max_seqlen, cudaStream_t stream);
+cudaError_t launch_bwd_dkdv(int d, const BwdParams& p, int max_seqlen, cudaStream_t stream);
+size_t bwd_smem_bytes(int d);
 
 cudaError_t launch_timeout_probe(uint32_t* status, unsigned long long limit_ns, cudaStream_t stream);
 
