@@ -443,12 +443,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             if (need_mask) {
                 const int hi = pos - kbase;                                          // keep column c <= hi
                 const int lo = (MODE == kModeLocal) ? pos - W + 1 - kbase : INT_MIN;  // keep column c >= lo
+                // Selects, not branches: a per-element branch costs more than the exponentials.
                 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int col = c * 32 + e;
-                        if (col > hi || col < lo) sr[c][e] = __float_as_uint(-INFINITY);
+                        sr[c][e] = (col <= hi) & (col >= lo) ? sr[c][e] : __float_as_uint(-INFINITY);
                     }
                 }
             }

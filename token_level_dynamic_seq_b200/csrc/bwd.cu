@@ -44,6 +44,7 @@
 
 #include <climits>
 #include <cstdint>
+#include <type_traits>
 
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -472,14 +473,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             const bool need_mask = (kbase + 63 > w.min_pos) || (MODE == kModeLocal && kbase < w.max_pos - W + 1);
             const int hi = pos - kbase;
             const int lo = (MODE == kModeLocal) ? pos - W + 1 - kbase : INT_MIN;
-            #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            // P = exp2(S * scale * log2(e) - lse); the mask as selects behind a uniform test.
+            if (need_mask) {
                 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int col = c * 32 + e;
-                    float x = fmaf(__uint_as_float(sr[c][e]), sl2, -lse2);
-                    if (need_mask && (col > hi || col < lo)) x = -INFINITY;
-                    sr[c][e] = __float_as_uint(fast_exp2(x));
+                for (int c = 0; c < 2; ++c) {
+                    #pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int col = c * 32 + e;
+                        const float x = fmaf(__uint_as_float(sr[c][e]), sl2, -lse2);
+                        sr[c][e] = __float_as_uint(fast_exp2((col <= hi) & (col >= lo) ? x : -INFINITY));
+                    }
+                }
+            } else {
+                #pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    #pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        sr[c][e] = __float_as_uint(fast_exp2(fmaf(__uint_as_float(sr[c][e]), sl2, -lse2)));
                 }
             }
             ok = __all_sync(0xffffffffu, mbar_wait(dp_full, j & 1, abort_flag, p.status, limit));
@@ -586,7 +596,7 @@ struct KvGeo {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_constant__ BwdParams p)
+__global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const __grid_constant__ BwdParams p)
 {
     using Geo = KvGeo<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -598,7 +608,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
     int* scol = reinterpret_cast<int*>(smem + Geo::kColOff);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Geo::kBarOff);
     uint64_t* kv_full = bars;
-    uint64_t* qd_full = kv_full + 1;   // [2], 32 arrivals (producer lanes) + bytes
+    uint64_t* qd_full = kv_full + 1;   // [2], 33 arrivals (producer lanes) + bytes
     uint64_t* qd_empty = qd_full + 2;  // [2]
     uint64_t* s_full = qd_empty + 2;
     uint64_t* dp_full = s_full + 1;
@@ -663,7 +673,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&qd_full[s], 32);
+            mbar_init(&qd_full[s], 33);  // lane 0's expect-tx arrival + one per producer lane after its stores
             mbar_init(&qd_empty[s], 1);
         }
         mbar_init(s_full, 1);
@@ -706,31 +716,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
             const int m = n % per_head;
             const bool local = m < nl;
             const int q0 = local ? j0 + 128 * m : r_start + 128 * (m - nl);  // position, or row of the list
-            int* cpos = scol + st * 384;
-            float* clse = reinterpret_cast<float*>(cpos + 128);
-            float* cdd = reinterpret_cast<float*>(cpos + 256);
-            #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int c = lane * 4 + u;
-                int qp = 0;
-                float l2 = INFINITY, dd = 0.f;
-                if (local) {
-                    qp = q0 + c;
-                    if (qp < len) {
-                        const size_t idx = ((size_t)(b * p.Hq + h)) * p.L + s0 + qp;
-                        l2 = p.lse[idx];
-                        dd = p.dl[idx];
-                    }
-                } else if (q0 + c < k_sel) {
-                    qp = p.sel_idx[sel_base + q0 + c];
-                    const size_t idx = (size_t)h * p.sel_stride + sel_base + q0 + c;
-                    l2 = p.lse_s[idx];
-                    dd = p.ds_sel[idx];
-                }
-                cpos[c] = qp;
-                clse[c] = l2;
-                cdd[c] = dd;
-            }
+            // Tile loads first: they do not depend on the column data, whose global loads
+            // then overlap the copies.
             if (lane == 0) {
                 mbar_arrive_expect_tx(&qd_full[st], 2 * Geo::kTile);
                 const CUtensorMap* mq = local ? &p.tm_q : &p.tm_qs;
@@ -742,9 +729,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                     tma_load_3d(sDo + st * Geo::kTile + c * Geo::kChunkBytes, mdo, &qd_full[st], c * 64, row, slab,
                                 pol_q);
                 }
-            } else {
-                mbar_arrive(&qd_full[st]);
             }
+            int* cpos = scol + st * 384;
+            float* clse = reinterpret_cast<float*>(cpos + 128);
+            float* cdd = reinterpret_cast<float*>(cpos + 256);
+            int qp[4];
+            float l2[4], dd[4];
+            #pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int c = lane * 4 + u;
+                qp[u] = 0;
+                l2[u] = INFINITY;
+                dd[u] = 0.f;
+                if (local) {
+                    qp[u] = q0 + c;
+                    if (qp[u] < len) {
+                        const size_t idx = ((size_t)(b * p.Hq + h)) * p.L + s0 + qp[u];
+                        l2[u] = __ldg(p.lse + idx);
+                        dd[u] = __ldg(p.dl + idx);
+                    }
+                } else if (q0 + c < k_sel) {
+                    qp[u] = __ldg(p.sel_idx + sel_base + q0 + c);
+                    const size_t idx = (size_t)h * p.sel_stride + sel_base + q0 + c;
+                    l2[u] = __ldg(p.lse_s + idx);
+                    dd[u] = __ldg(p.ds_sel + idx);
+                }
+            }
+            *reinterpret_cast<int4*>(cpos + lane * 4) = make_int4(qp[0], qp[1], qp[2], qp[3]);
+            *reinterpret_cast<float4*>(clse + lane * 4) = make_float4(l2[0], l2[1], l2[2], l2[3]);
+            *reinterpret_cast<float4*>(cdd + lane * 4) = make_float4(dd[0], dd[1], dd[2], dd[3]);
+            mbar_arrive(&qd_full[st]);  // every lane, after its column stores
             ++issued;
         }
         if (lane == 0) {
@@ -851,21 +865,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
             const int q_first = cpos[0 - 64 * half];
             const int q_last = local ? q_first + 127 : INT_MAX;
             const bool need_mask = !(q_first >= j0 + 127 && (!local || q_last - j0 < W));
-            #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            const int wl = local ? W : INT_MAX;  // a query more than wl - 1 past the key is out
+            // P^T = exp2(S^T * scale * log2(e) - lse(query)); the mask, where the tile needs it,
+            // as selects (a per-element branch here costs more than the exponentials).
+            auto p_chunk = [&](int c, auto masked) {
                 uint32_t pk[16];
                 #pragma unroll
                 for (int e4 = 0; e4 < 32; e4 += 4) {
                     const int col = c * 32 + e4;
                     const float4 l4 = *reinterpret_cast<const float4*>(clse + col);
                     const float la[4] = {l4.x, l4.y, l4.z, l4.w};
-                    int4 q4 = make_int4(0, 0, 0, 0);
-                    if (need_mask) q4 = *reinterpret_cast<const int4*>(cpos + col);
-                    const int qa[4] = {q4.x, q4.y, q4.z, q4.w};
+                    int qa[4] = {0, 0, 0, 0};
+                    if (decltype(masked)::value) {
+                        const int4 q4 = *reinterpret_cast<const int4*>(cpos + col);
+                        qa[0] = q4.x;
+                        qa[1] = q4.y;
+                        qa[2] = q4.z;
+                        qa[3] = q4.w;
+                    }
                     #pragma unroll
                     for (int t = 0; t < 4; ++t) {
                         float x = fmaf(__uint_as_float(sr[c][e4 + t]), sl2, -la[t]);
-                        if (need_mask && (qa[t] < kp || (local && qa[t] - kp >= W))) x = -INFINITY;
+                        if (decltype(masked)::value) {
+                            const int dq = qa[t] - kp;
+                            x = (dq >= 0) & (dq < wl) ? x : -INFINITY;
+                        }
                         sr[c][e4 + t] = __float_as_uint(fast_exp2(x));
                     }
                 }
@@ -873,6 +897,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                 for (int e = 0; e < 32; e += 2)
                     pk[e / 2] = pack_bf16x2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
                 tmem_st16(tS + 16 * c, pk);  // P^T over S^T columns already read
+            };
+            if (need_mask) {
+                p_chunk(0, std::true_type{});
+                p_chunk(1, std::true_type{});
+            } else {
+                p_chunk(0, std::false_type{});
+                p_chunk(1, std::false_type{});
             }
             tmem_wait_st();
             tc_fence_before();
