@@ -282,7 +282,9 @@ def run_train(args, rank, world):
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
-    w = workloads.load("c32k", seed=rank)
+    base = args.workload[len("train_"):]
+    w = workloads.load(base, seed=rank)
+    assert w.cu_seqlens is None, "the training bench takes fixed-length workloads"
     q, k, v, g = w.q.to(dev), w.k.to(dev), w.v.to(dev), w.g.to(dev)
     gen = torch.Generator(device=dev)
     gen.manual_seed(1000 + rank)
@@ -330,12 +332,14 @@ def run_train(args, rank, world):
     achieved = bwd_flops / (bwd_ms * 1e-3) / 1e12
     tokens = sum(w.seqlens)
     line = {
-        "metric": "LoGo training step tokens/s (forward + backward, 32K tokens, 20% global)",
+        "metric": f"LoGo training step tokens/s (forward + backward, {base})",
         "value": tokens / (total_ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "train_c32k", "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "d": w.d, "W": w.W,
-                   "ratio": w.ratio, "selected": tot_sel, "l2": "inputs (Q 268 MB) larger than L2"},
+        "config": {"workload": args.workload, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "d": w.d, "W": w.W,
+                   "ratio": w.ratio, "selected": tot_sel,
+                   "l2": f"inputs (Q {q.numel() * 2 / 1e6:.0f} MB) " + ("larger" if q.numel() * 2 > 126e6 else "smaller")
+                         + " than L2"},
         "forward_ms": fwd_ms, "backward_ms": bwd_ms,
         "backward_useful_tflops": achieved, "backward_executed_tflops": bwd_exec / (bwd_ms * 1e-3) / 1e12,
         "roofline": {"kernel": "backward (prep, dQ selected, dQ local, dK/dV)", "bound": "tensor",
@@ -358,7 +362,7 @@ def main():
     if args.workload == "decode_c32k":
         run_decode(args, rank, world)
         return
-    if args.workload == "train_c32k":
+    if args.workload.startswith("train_"):
         run_train(args, rank, world)
         return
     assert args.warmup >= 3, "at least 3 warm-up steps"

@@ -577,6 +577,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
 
 // ------------------------------------------------------------------ dK, dV
 
+constexpr int kKvThreads = kBwdThreads + 32;  // + one warp that stages the per-column data
+constexpr int kColStages = 4;                  // column data runs up to four query tiles ahead
+
 template <int D>
 struct KvGeo {
     static constexpr int kChunkBytes = 128 * 128;
@@ -585,9 +588,9 @@ struct KvGeo {
     static constexpr int kVOff = kTile;
     static constexpr int kQOff = 2 * kTile;             // [2] query tiles
     static constexpr int kDoOff = kQOff + 2 * kTile;    // [2] dout tiles
-    static constexpr int kColOff = kDoOff + 2 * kTile;  // [2][3][128]: position, lse, D per column
-    static constexpr int kBarOff = kColOff + 2 * 3 * 128 * 4;
-    static constexpr int kNumBars = 1 + 2 + 2 + 1 + 1 + 1 + 1 + 1 + 1;
+    static constexpr int kColOff = kDoOff + 2 * kTile;  // [kColStages][3][128]: position, lse, D per column
+    static constexpr int kBarOff = kColOff + kColStages * 3 * 128 * 4;
+    static constexpr int kNumBars = 1 + 2 * 4 + 2 * kColStages + 6;
     static constexpr int kBytes = kBarOff + kNumBars * 8 + 16 + 16;
     static constexpr uint32_t kTmemS = 0;    // S^T, overwritten in place by P^T (bf16)
     static constexpr uint32_t kTmemDP = 128; // dP^T, overwritten in place by dS^T
@@ -595,8 +598,11 @@ struct KvGeo {
     static constexpr uint32_t kTmemDK = 256 + D;
 };
 
+// Warp roles: 0 TMA (K, V once; Q and dout tiles), 1 tcgen05 issuer, 2-9 softmax (two
+// warpgroups, one per half of the 128 query columns), 10 per-column data (query position,
+// log-sum-exp, D) into a ring of kColStages slots, so those loads never gate the copies.
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const __grid_constant__ BwdParams p)
+__global__ void __launch_bounds__(kKvThreads) bwd_dkdv_kernel(const __grid_constant__ BwdParams p)
 {
     using Geo = KvGeo<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -608,9 +614,13 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const __grid_cons
     int* scol = reinterpret_cast<int*>(smem + Geo::kColOff);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Geo::kBarOff);
     uint64_t* kv_full = bars;
-    uint64_t* qd_full = kv_full + 1;   // [2], 33 arrivals (producer lanes) + bytes
-    uint64_t* qd_empty = qd_full + 2;  // [2]
-    uint64_t* s_full = qd_empty + 2;
+    uint64_t* q_full = kv_full + 1;     // [2]
+    uint64_t* q_empty = q_full + 2;     // [2]: after dK of the tile
+    uint64_t* do_full = q_empty + 2;    // [2]
+    uint64_t* do_empty = do_full + 2;   // [2]: after dV of the tile
+    uint64_t* col_full = do_empty + 2;  // [kColStages], 32 arrivals
+    uint64_t* col_empty = col_full + kColStages;  // [kColStages], 256 arrivals
+    uint64_t* s_full = col_empty + kColStages;
     uint64_t* dp_full = s_full + 1;
     uint64_t* p_full = dp_full + 1;    // 256 arrivals
     uint64_t* ds_full = p_full + 1;    // 256 arrivals
@@ -673,8 +683,14 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const __grid_cons
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&qd_full[s], 33);  // lane 0's expect-tx arrival + one per producer lane after its stores
-            mbar_init(&qd_empty[s], 1);
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
+            mbar_init(&do_full[s], 1);
+            mbar_init(&do_empty[s], 1);
+        }
+        for (int s = 0; s < kColStages; ++s) {
+            mbar_init(&col_full[s], 32);
+            mbar_init(&col_empty[s], 256);
         }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
@@ -696,43 +712,65 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const __grid_cons
     const uint64_t limit = p.timeout_ns;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer: K, V once; Q, dO and column data per tile
-        const uint64_t pol_kv = policy_evict_first();
-        const uint64_t pol_q = policy_evict_last();
+        // ------------------------------------------------------------ TMA: K, V once; Q and dout per tile
         if (lane == 0) {
+            const uint64_t pol_kv = policy_evict_first();
+            const uint64_t pol_q = policy_evict_last();
             mbar_arrive_expect_tx(kv_full, 2 * Geo::kTile);
             for (int c = 0; c < D / 64; ++c) {
                 tma_load_3d(sK + c * Geo::kChunkBytes, &p.tm_k, kv_full, c * 64, s0 + j0, zkv, pol_kv);
                 tma_load_3d(sV + c * Geo::kChunkBytes, &p.tm_v, kv_full, c * 64, s0 + j0, zkv, pol_kv);
             }
+            bool ok = true;
+            int nq = 0, ndo = 0;  // tiles whose copies were started
+            for (int n = 0; n < nb && ok; ++n) {
+                const int st = n & 1;
+                const int h = hk * p.G + n / per_head;
+                const int m = n % per_head;
+                const bool local = m < nl;
+                const int q0 = local ? j0 + 128 * m : r_start + 128 * (m - nl);
+                const int row = local ? s0 + q0 : sel_base + q0;
+                const int slab = local ? b * p.Hq + h : h;
+                // dout of tile n - 2 is released after its dV, before its Q (after dK): copy dout first.
+                if (n >= 2) ok = mbar_wait(&do_empty[st], ((n >> 1) - 1) & 1, abort_flag, p.status, limit);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&do_full[st], Geo::kTile);
+                ++ndo;
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_3d(sDo + st * Geo::kTile + c * Geo::kChunkBytes, local ? &p.tm_do : &p.tm_dos,
+                                &do_full[st], c * 64, row, slab, pol_q);
+                if (n >= 2) ok = mbar_wait(&q_empty[st], ((n >> 1) - 1) & 1, abort_flag, p.status, limit);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&q_full[st], Geo::kTile);
+                ++nq;
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_3d(sQ + st * Geo::kTile + c * Geo::kChunkBytes, local ? &p.tm_q : &p.tm_qs,
+                                &q_full[st], c * 64, row, slab, pol_q);
+            }
+            volatile int dummy = 0;
+            if (*abort_flag) {
+                // stage s was filled (count - s + 1) / 2 times; wait for its last fill
+                for (int s = 0; s < 2 && s < nq; ++s)
+                    mbar_wait(&q_full[s], ((nq - s + 1) / 2 - 1) & 1, &dummy, nullptr, limit);
+                for (int s = 0; s < 2 && s < ndo; ++s)
+                    mbar_wait(&do_full[s], ((ndo - s + 1) / 2 - 1) & 1, &dummy, nullptr, limit);
+            }
+            // K and V always land before the CTA ends (the MMA thread may have given up first).
+            mbar_wait(kv_full, 0, &dummy, nullptr, limit);
         }
+    } else if (warp == 10) {
+        // ------------------------------------------------------------ per-column data ring
         bool ok = true;
-        int issued = 0;  // query tiles whose loads were started
         for (int n = 0; n < nb && ok; ++n) {
-            const int st = n & 1;
-            if (n >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&qd_empty[st], ((n >> 1) - 1) & 1, abort_flag, p.status, limit));
+            const int cs = n % kColStages;
+            if (n >= kColStages)
+                ok = __all_sync(0xffffffffu, mbar_wait(&col_empty[cs], ((n / kColStages) - 1) & 1, abort_flag,
+                                                       p.status, limit));
             if (!ok) break;
             const int h = hk * p.G + n / per_head;
             const int m = n % per_head;
             const bool local = m < nl;
-            const int q0 = local ? j0 + 128 * m : r_start + 128 * (m - nl);  // position, or row of the list
-            // Tile loads first: they do not depend on the column data, whose global loads
-            // then overlap the copies.
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&qd_full[st], 2 * Geo::kTile);
-                const CUtensorMap* mq = local ? &p.tm_q : &p.tm_qs;
-                const CUtensorMap* mdo = local ? &p.tm_do : &p.tm_dos;
-                const int row = local ? s0 + q0 : sel_base + q0;
-                const int slab = local ? b * p.Hq + h : h;
-                for (int c = 0; c < D / 64; ++c) {
-                    tma_load_3d(sQ + st * Geo::kTile + c * Geo::kChunkBytes, mq, &qd_full[st], c * 64, row, slab, pol_q);
-                    tma_load_3d(sDo + st * Geo::kTile + c * Geo::kChunkBytes, mdo, &qd_full[st], c * 64, row, slab,
-                                pol_q);
-                }
-            }
-            int* cpos = scol + st * 384;
-            float* clse = reinterpret_cast<float*>(cpos + 128);
-            float* cdd = reinterpret_cast<float*>(cpos + 256);
+            const int q0 = local ? j0 + 128 * m : r_start + 128 * (m - nl);
             int qp[4];
             float l2[4], dd[4];
             #pragma unroll
@@ -755,20 +793,11 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const __grid_cons
                     dd[u] = __ldg(p.ds_sel + idx);
                 }
             }
+            int* cpos = scol + cs * 384;
             *reinterpret_cast<int4*>(cpos + lane * 4) = make_int4(qp[0], qp[1], qp[2], qp[3]);
-            *reinterpret_cast<float4*>(clse + lane * 4) = make_float4(l2[0], l2[1], l2[2], l2[3]);
-            *reinterpret_cast<float4*>(cdd + lane * 4) = make_float4(dd[0], dd[1], dd[2], dd[3]);
-            mbar_arrive(&qd_full[st]);  // every lane, after its column stores
-            ++issued;
-        }
-        if (lane == 0) {
-            volatile int dummy = 0;
-            if (*abort_flag) {
-                for (int s = 0; s < 2 && s < issued; ++s)
-                    mbar_wait(&qd_full[s], ((issued - s + 1) / 2 - 1) & 1, &dummy, nullptr, limit);
-            }
-            // K and V always land before the CTA ends (the MMA thread may have given up first).
-            mbar_wait(kv_full, 0, &dummy, nullptr, limit);
+            *reinterpret_cast<float4*>(cpos + 128 + lane * 4) = make_float4(l2[0], l2[1], l2[2], l2[3]);
+            *reinterpret_cast<float4*>(cpos + 256 + lane * 4) = make_float4(dd[0], dd[1], dd[2], dd[3]);
+            mbar_arrive(&col_full[cs]);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ tcgen05 issuer
@@ -794,23 +823,28 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const __grid_cons
                 }
             };
             bool ok = mbar_wait(kv_full, 0, abort_flag, p.status, limit);
-            if (ok) ok = mbar_wait(&qd_full[0], 0, abort_flag, p.status, limit);
+            if (ok) ok = mbar_wait(&q_full[0], 0, abort_flag, p.status, limit);
             if (ok) {
                 tc_fence_after();
                 issue_kmajor(tmem + Geo::kTmemS, sKa, sQa);
                 umma_commit(s_full);
+                ok = mbar_wait(&do_full[0], 0, abort_flag, p.status, limit);
+            }
+            if (ok) {
+                tc_fence_after();
                 issue_kmajor(tmem + Geo::kTmemDP, sVa, sDoa);
                 umma_commit(dp_full);
             }
             for (int n = 0; n < nb && ok; ++n) {
                 const int st = n & 1;
+                const bool nxt = n + 1 < nb;
                 ok = mbar_wait(p_full, n & 1, abort_flag, p.status, limit);
                 if (!ok) break;
                 tc_fence_after();
                 issue_acc(tmem + Geo::kTmemDV, tmem + Geo::kTmemS, sDoa + st * Geo::kTile, n == 0);
-                const bool nxt = n + 1 < nb;
+                umma_commit(&do_empty[st]);
                 if (nxt) {
-                    ok = mbar_wait(&qd_full[st ^ 1], ((n + 1) >> 1) & 1, abort_flag, p.status, limit);
+                    ok = mbar_wait(&q_full[st ^ 1], ((n + 1) >> 1) & 1, abort_flag, p.status, limit);
                     if (!ok) break;
                     tc_fence_after();
                     issue_kmajor(tmem + Geo::kTmemS, sKa, sQa + (st ^ 1) * Geo::kTile);
@@ -820,8 +854,11 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const __grid_cons
                 if (!ok) break;
                 tc_fence_after();
                 issue_acc(tmem + Geo::kTmemDK, tmem + Geo::kTmemDP, sQa + st * Geo::kTile, n == 0);
-                umma_commit(&qd_empty[st]);
+                umma_commit(&q_empty[st]);
                 if (nxt) {
+                    ok = mbar_wait(&do_full[st ^ 1], ((n + 1) >> 1) & 1, abort_flag, p.status, limit);
+                    if (!ok) break;
+                    tc_fence_after();
                     issue_kmajor(tmem + Geo::kTmemDP, sVa, sDoa + (st ^ 1) * Geo::kTile);
                     umma_commit(dp_full);
                 }
@@ -842,16 +879,13 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const __grid_cons
         const int W = p.window;
         bool ok = true;
         for (int n = 0; n < nb; ++n) {
-            const int st = n & 1;
+            const int cs = n % kColStages;
             const int m = n % per_head;
             const bool local = m < nl;
-            const int* cpos = scol + st * 384 + 64 * half;
-            const float* clse = reinterpret_cast<const float*>(scol + st * 384 + 128 + 64 * half);
-            const float* cdd = reinterpret_cast<const float*>(scol + st * 384 + 256 + 64 * half);
-            // The column data of this tile was published on qd_full; that phase has completed
-            // (the MMA for this tile waited on it) and cannot advance before this tile's dS
-            // is in, so this wait returns at once and orders the reads after the producer's writes.
-            ok = __all_sync(0xffffffffu, mbar_wait(&qd_full[st], (n >> 1) & 1, abort_flag, p.status, limit));
+            const int* cpos = scol + cs * 384 + 64 * half;
+            const float* clse = reinterpret_cast<const float*>(scol + cs * 384 + 128 + 64 * half);
+            const float* cdd = reinterpret_cast<const float*>(scol + cs * 384 + 256 + 64 * half);
+            ok = __all_sync(0xffffffffu, mbar_wait(&col_full[cs], (n / kColStages) & 1, abort_flag, p.status, limit));
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full, n & 1, abort_flag, p.status, limit));
             if (!ok) break;
             tc_fence_after();
@@ -934,6 +968,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const __grid_cons
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(ds_full);
+            mbar_arrive(&col_empty[cs]);  // this tile's column data has been read
         }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.status, limit));
         if (ok) {
@@ -976,11 +1011,12 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const __grid_cons
 }
 
 template <typename K>
-cudaError_t launch_big(K kern, size_t smem, dim3 grid, const BwdParams& p, cudaStream_t stream)
+cudaError_t launch_big(K kern, size_t smem, dim3 grid, const BwdParams& p, cudaStream_t stream,
+                       int threads = kBwdThreads)
 {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kBwdThreads, smem, stream>>>(p);
+    kern<<<grid, threads, smem, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -1026,8 +1062,8 @@ cudaError_t launch_bwd_dkdv(int d, const BwdParams& p, int max_seqlen, cudaStrea
 {
     const dim3 grid((max_seqlen + 127) / 128, p.Hkv, p.nseq);
     if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
-    if (d == 64) return launch_big(bwd_dkdv_kernel<64>, KvGeo<64>::kBytes + 1024, grid, p, stream);
-    return launch_big(bwd_dkdv_kernel<128>, KvGeo<128>::kBytes + 1024, grid, p, stream);
+    if (d == 64) return launch_big(bwd_dkdv_kernel<64>, KvGeo<64>::kBytes + 1024, grid, p, stream, kKvThreads);
+    return launch_big(bwd_dkdv_kernel<128>, KvGeo<128>::kBytes + 1024, grid, p, stream, kKvThreads);
 }
 
 size_t bwd_smem_bytes(int d)
