@@ -44,6 +44,9 @@ def parse():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", default="sequences", choices=["sequences", "heads"],
+                    help="sequences: each rank runs its own sequence (weak scaling); heads: the ranks split one "
+                         "problem by key/value-head groups (strong scaling)")
     return ap.parse_args()
 
 
@@ -376,8 +379,15 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
-    w = workloads.load(args.workload, seed=rank)
-    q, k, v, g = w.q.to(dev), w.k.to(dev), w.v.to(dev), w.g.to(dev)
+    by_heads = args.shard == "heads"
+    w = workloads.load(args.workload, seed=0 if by_heads else rank)
+    hq, hk, hv = w.q, w.k, w.v
+    if by_heads:
+        # every rank holds the whole (tiny) gate and recomputes the same selection
+        assert world <= w.Hkv, "head sharding needs at least one key/value head per rank"
+        hq, hk, hv = multirank.head_slice(w.q, w.k, w.v, multirank.shard_heads(w.Hq, w.Hkv, world)[rank])
+    q, k, v, g = hq.to(dev), hk.to(dev), hv.to(dev), w.g.to(dev)
+    Hq_r = q.shape[1]
     cu = None if w.cu_seqlens is None else w.cu_seqlens.to(dev)
     ml = max(w.seqlens)
     shape = logo.make_shape(q, k, cu, ml)
@@ -412,8 +422,8 @@ def main():
     tot_sel = int(cu_sel[-1].item())
     sel_pos_sum = int(sel[:tot_sel].to(torch.int64).sum().item()) + tot_sel
     lp = sum(min(w.W, n) * (min(w.W, n) + 1) // 2 + (n - min(w.W, n)) * min(w.W, n) for n in w.seqlens)
-    fl_local = 4 * w.d * w.Hq * lp
-    fl_global = 4 * w.d * w.Hq * sel_pos_sum
+    fl_local = 4 * w.d * Hq_r * lp
+    fl_global = 4 * w.d * Hq_r * sel_pos_sum
     tokens = w.tokens
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
@@ -441,10 +451,11 @@ def main():
         per["global"].append(e[2].elapsed_time(e[3]))
     avg = {kk: sum(vv) / len(vv) for kk, vv in per.items()}
     ms_step = multirank.max_over_ranks(t_total_ms / args.steps, device=dev)  # slowest rank
-    job_tokens = int(multirank.sum_over_ranks(tokens, device=dev))
+    # head sharding: all ranks work on the same tokens; sequence sharding: on their own
+    job_tokens = tokens if by_heads else int(multirank.sum_over_ranks(tokens, device=dev))
 
     # end to end through the public API: pinned host inputs -> forward -> host output
-    pin = [x.pin_memory() for x in (w.q, w.k, w.v, w.g)]
+    pin = [x.contiguous().pin_memory() for x in (hq, hk, hv, w.g)]
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     h2d = sum(x.numel() * x.element_size() for x in pin)
     d2h = out_host.numel() * out_host.element_size()
@@ -490,12 +501,13 @@ def main():
             "warmup": args.warmup,
             "ms_per_step": ms_step,
             "higher_is_better": True,
-            "scaling": "weak",
+            "scaling": "strong" if by_heads else "weak",
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic",
             "config": {"workload": w.name, "desc": w.recipe, "tokens_per_rank": tokens,
-                       "parallelism": f"independent sequences x{world}",
+                       "parallelism": (f"key/value-head groups x{world}" if by_heads
+                                       else f"independent sequences x{world}"),
                        "l2": "inputs larger than L2 (Q+K+V+O = %.0f MB > 126 MB)" % (
                            (q.numel() + k.numel() + v.numel() + out.numel()) * 2 / 1e6)},
             "useful_tflops": useful_tflops,
