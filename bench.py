@@ -44,6 +44,7 @@ def parse():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-batch", type=int, default=64, help="sequences of the decode workload")
     ap.add_argument("--shard", default="sequences", choices=["sequences", "heads"],
                     help="sequences: each rank runs its own sequence (weak scaling); heads: the ranks split one "
                          "problem by key/value-head groups (strong scaling)")
@@ -222,7 +223,7 @@ def run_decode(args, rank, world):
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
-    B, Hq, Hkv, L, d, W, ratio = 64, 32, 8, 32768, 128, 4096, 0.2
+    B, Hq, Hkv, L, d, W, ratio = args.decode_batch, 32, 8, 32768, 128, 4096, 0.2
     gen = torch.Generator(device=dev)
     gen.manual_seed(rank)
     q = torch.randn(B, Hq, d, generator=gen, device=dev).to(torch.bfloat16)
@@ -260,11 +261,12 @@ def run_decode(args, rank, world):
     peak_burst, peak_sust, hbm, peak_src = peaks()
     achieved = bytes_step / (ms * 1e-3) / 1e9
     line = {
-        "metric": "LoGo decode tokens/s (64 x 32K caches, W=4096, ~20% global)", "value": B / (ms * 1e-3),
+        "metric": f"LoGo decode tokens/s ({B} x 32K caches, W=4096, ~20% global)", "value": B / (ms * 1e-3),
         "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": "decode_c32k", "B": B, "Hq": Hq, "Hkv": Hkv, "cache": L, "d": d, "W": W,
-                   "ratio": ratio, "selected": n_sel, "l2": "caches (8.6 GB) larger than L2"},
+                   "ratio": ratio, "selected": n_sel,
+                   "l2": f"caches ({kc.numel() * 4 / 1e9:.1f} GB) larger than L2"},
         "roofline": {"kernel": "decode_partial_kernel + decode_combine_kernel", "bound": "hbm",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
                      "peak_source": f"{peak_src} HBM copy bandwidth"},
