@@ -622,9 +622,9 @@ __global__ void __launch_bounds__(kKvThreads) bwd_dkdv_kernel(const __grid_const
     uint64_t* col_empty = col_full + kColStages;  // [kColStages], 256 arrivals
     uint64_t* s_full = col_empty + kColStages;
     uint64_t* dp_full = s_full + 1;
-    uint64_t* p_full = dp_full + 1;    // 256 arrivals
-    uint64_t* ds_full = p_full + 1;    // 256 arrivals
-    uint64_t* acc_full = ds_full + 1;
+    uint64_t* s_read = dp_full + 1;    // 256 arrivals: S^T of the tile is in registers, its columns are free
+    uint64_t* pd_full = s_read + 1;    // 256 arrivals: P^T and dS^T written over dP^T
+    uint64_t* acc_full = pd_full + 1;
     uint64_t* drain = acc_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -694,8 +694,8 @@ __global__ void __launch_bounds__(kKvThreads) bwd_dkdv_kernel(const __grid_const
         }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
-        mbar_init(p_full, 256);
-        mbar_init(ds_full, 256);
+        mbar_init(s_read, 256);
+        mbar_init(pd_full, 256);
         mbar_init(acc_full, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -813,11 +813,13 @@ __global__ void __launch_bounds__(kKvThreads) bwd_dkdv_kernel(const __grid_const
                             kk > 0 ? 1u : 0u);
                 }
             };
-            // acc += X^T-tile (bf16 in TMEM, queries 0-63 in columns 0-31, 64-127 in 64-95) times a [128 x D] tile.
-            auto issue_acc = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, bool first) {
+            // acc += X^T-tile (bf16 in the dP^T columns) times a [128 x D] tile.  Queries 32c .. 32c+31
+            // of warpgroup h sit in columns 64h + 32c + which * 16 .. +15 (which 0: P^T, 1: dS^T).
+            auto issue_acc = [&](uint32_t d_tmem, int which, uint32_t b_base, bool first) {
                 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t a = a_tmem + (kk >> 2) * 64 + (kk & 3) * 8;
+                    const uint32_t a = tmem + Geo::kTmemDP + (kk >> 2) * 64 + ((kk >> 1) & 1) * 32 + which * 16 +
+                                       (kk & 1) * 8;
                     const uint64_t bd = sdesc_sw128(b_base + kk * 2048, Geo::kChunkBytes, 1024);
                     umma_ts(d_tmem, a, bd, idesc_acc, (!first || kk > 0) ? 1u : 0u);
                 }
@@ -835,25 +837,26 @@ __global__ void __launch_bounds__(kKvThreads) bwd_dkdv_kernel(const __grid_const
                 issue_kmajor(tmem + Geo::kTmemDP, sVa, sDoa);
                 umma_commit(dp_full);
             }
+            // Per tile n: S^T(n+1) as soon as the softmax has read S^T(n); dV(n), dK(n) once P^T(n)
+            // and dS^T(n) are in the dP^T columns; then dP^T(n+1) over them (tcgen05 MMAs from one
+            // thread execute in issue order, so it writes only after dV(n) and dK(n) have read).
             for (int n = 0; n < nb && ok; ++n) {
                 const int st = n & 1;
                 const bool nxt = n + 1 < nb;
-                ok = mbar_wait(p_full, n & 1, abort_flag, p.status, limit);
-                if (!ok) break;
-                tc_fence_after();
-                issue_acc(tmem + Geo::kTmemDV, tmem + Geo::kTmemS, sDoa + st * Geo::kTile, n == 0);
-                umma_commit(&do_empty[st]);
                 if (nxt) {
-                    ok = mbar_wait(&q_full[st ^ 1], ((n + 1) >> 1) & 1, abort_flag, p.status, limit);
+                    ok = mbar_wait(s_read, n & 1, abort_flag, p.status, limit);
+                    if (ok) ok = mbar_wait(&q_full[st ^ 1], ((n + 1) >> 1) & 1, abort_flag, p.status, limit);
                     if (!ok) break;
                     tc_fence_after();
                     issue_kmajor(tmem + Geo::kTmemS, sKa, sQa + (st ^ 1) * Geo::kTile);
                     umma_commit(s_full);
                 }
-                ok = mbar_wait(ds_full, n & 1, abort_flag, p.status, limit);
+                ok = mbar_wait(pd_full, n & 1, abort_flag, p.status, limit);
                 if (!ok) break;
                 tc_fence_after();
-                issue_acc(tmem + Geo::kTmemDK, tmem + Geo::kTmemDP, sQa + st * Geo::kTile, n == 0);
+                issue_acc(tmem + Geo::kTmemDV, 0, sDoa + st * Geo::kTile, n == 0);
+                umma_commit(&do_empty[st]);
+                issue_acc(tmem + Geo::kTmemDK, 1, sQa + st * Geo::kTile, n == 0);
                 umma_commit(&q_empty[st]);
                 if (nxt) {
                     ok = mbar_wait(&do_full[st ^ 1], ((n + 1) >> 1) & 1, abort_flag, p.status, limit);
@@ -895,6 +898,9 @@ __global__ void __launch_bounds__(kKvThreads) bwd_dkdv_kernel(const __grid_const
             tmem_ld32(tS + 32, sr[1]);
             tmem_wait_ld(sr[0]);
             tmem_wait_ld(sr[1]);
+            // S^T is in registers: the next tile's S^T may go into these columns now.
+            tc_fence_before();
+            mbar_arrive(s_read);
             // Tile-wide test: every (key, query) pair of the tile inside the mask.
             const int q_first = cpos[0 - 64 * half];
             const int q_last = local ? q_first + 127 : INT_MAX;
@@ -903,7 +909,6 @@ __global__ void __launch_bounds__(kKvThreads) bwd_dkdv_kernel(const __grid_const
             // P^T = exp2(S^T * scale * log2(e) - lse(query)); the mask, where the tile needs it,
             // as selects (a per-element branch here costs more than the exponentials).
             auto p_chunk = [&](int c, auto masked) {
-                uint32_t pk[16];
                 #pragma unroll
                 for (int e4 = 0; e4 < 32; e4 += 4) {
                     const int col = c * 32 + e4;
@@ -927,10 +932,6 @@ __global__ void __launch_bounds__(kKvThreads) bwd_dkdv_kernel(const __grid_const
                         sr[c][e4 + t] = __float_as_uint(fast_exp2(x));
                     }
                 }
-                #pragma unroll
-                for (int e = 0; e < 32; e += 2)
-                    pk[e / 2] = pack_bf16x2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
-                tmem_st16(tS + 16 * c, pk);  // P^T over S^T columns already read
             };
             if (need_mask) {
                 p_chunk(0, std::true_type{});
@@ -939,19 +940,18 @@ __global__ void __launch_bounds__(kKvThreads) bwd_dkdv_kernel(const __grid_const
                 p_chunk(0, std::false_type{});
                 p_chunk(1, std::false_type{});
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(p_full);
             ok = __all_sync(0xffffffffu, mbar_wait(dp_full, n & 1, abort_flag, p.status, limit));
             if (!ok) break;
             tc_fence_after();
             const uint32_t tD = tmem + lane_off + Geo::kTmemDP + 64 * half;
             #pragma unroll
             for (int c = 0; c < 2; ++c) {
+                // dP^T columns 32c .. 32c+31 of this warpgroup, then P^T and dS^T of the same
+                // 32 queries over exactly those columns (16 each).
                 uint32_t dp[32];
                 tmem_ld32(tD + 32 * c, dp);
                 tmem_wait_ld(dp);
-                uint32_t pk[16];
+                uint32_t pp[16], pk[16];
                 #pragma unroll
                 for (int e4 = 0; e4 < 32; e4 += 4) {
                     const float4 d4 = *reinterpret_cast<const float4*>(cdd + c * 32 + e4);
@@ -962,12 +962,15 @@ __global__ void __launch_bounds__(kKvThreads) bwd_dkdv_kernel(const __grid_const
                         ds[t] = __uint_as_float(sr[c][e4 + t]) * (__uint_as_float(dp[e4 + t]) - da[t]);
                     pk[e4 / 2] = pack_bf16x2(ds[0], ds[1]);
                     pk[e4 / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+                    pp[e4 / 2] = pack_bf16x2(__uint_as_float(sr[c][e4]), __uint_as_float(sr[c][e4 + 1]));
+                    pp[e4 / 2 + 1] = pack_bf16x2(__uint_as_float(sr[c][e4 + 2]), __uint_as_float(sr[c][e4 + 3]));
                 }
-                tmem_st16(tD + 16 * c, pk);
+                tmem_st16(tD + 32 * c, pp);
+                tmem_st16(tD + 32 * c + 16, pk);
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(ds_full);
+            mbar_arrive(pd_full);
             mbar_arrive(&col_empty[cs]);  // this tile's column data has been read
         }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.status, limit));
