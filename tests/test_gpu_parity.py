@@ -22,13 +22,13 @@ MAX_ABS = 2e-2
 REL_L2 = 5e-3
 
 
-def close(got, ref, what=""):
+def close(got, ref, what="", max_abs=MAX_ABS):
     got = got.double().cpu()
     ref = ref.double().cpu()
     assert torch.isfinite(got).all(), f"{what}: non-finite output"
     err = (got - ref).abs().max().item()
     rel = ((got - ref).norm() / ref.norm().clamp_min(1e-30)).item()
-    assert err <= MAX_ABS and rel <= REL_L2, f"{what}: max-abs {err:.3e}, rel-L2 {rel:.3e}"
+    assert err <= max_abs and rel <= REL_L2, f"{what}: max-abs {err:.3e} (bound {max_abs:.3e}), rel-L2 {rel:.3e}"
     return err, rel
 
 
@@ -120,6 +120,71 @@ def test_forward_small_full(case):
         mask[bi, ti] = False
         untouched = sentinel.cpu().permute(0, 2, 1, 3)[mask]
         assert (untouched == 7.0).all()
+
+
+RESCALE = [
+    # name, B, Hq, Hkv, L, d, W, ratio, kind
+    ("ramp d128", 1, 4, 2, 1500, 128, 700, 0.2, "ramp"),
+    ("spikes d128", 1, 4, 2, 1300, 128, 1300, 0.3, "spikes"),
+    ("ramp d64 g1", 2, 2, 2, 900, 64, 400, 0.25, "ramp"),
+]
+
+
+@pytest.mark.parametrize("case", RESCALE, ids=[c[0] for c in RESCALE])
+def test_forward_running_max_growth(case):
+    """Rows whose running maximum grows past the rescale threshold on later key tiles.
+
+    With N(0,1) inputs the maximum of a row settles within the first key tile,
+    so the online softmax's rescale step would only ever run there.  Here key
+    norms grow along the sequence (ramp: x1 at the start to x9 at the end) or a
+    few keys carry a large norm (spikes: every 97th key x12), so the maximum
+    keeps growing by many powers of two from tile to tile.
+
+    Outputs here reach |o| ~ 8, where one bf16 rounding alone is up to 2^-6
+    (0.016) and the merged output is rounded twice (the local branch is stored
+    in bf16 and read back by the merge), so an absolute 2e-2 bound is finer
+    than the output format at that magnitude (a CPU emulation of the rounding
+    steps alone gives 0.021 to 0.027).  The max-abs bound is therefore scaled
+    with the output: 2e-2 * max(1, max|ref| / 4), i.e. 2e-2 at the magnitude
+    of N(0,1) outputs; the relative-L2 bound stays 5e-3.
+    """
+    name, B, Hq, Hkv, L, d, W, ratio, kind = case
+    w = workloads.make(B, Hq, Hkv, L, d, W, ratio, seed=5, qkv_scale=1.0, name=name)
+    if kind == "ramp":
+        f = 1.0 + 8.0 * torch.arange(L, dtype=torch.float32) / L
+    else:
+        f = torch.ones(L)
+        f[::97] = 12.0
+    w.k = (w.k.float() * f[None, None, :, None]).bfloat16()
+    q, k, v, g, cu = to_dev(w)
+    ws = logo.workspace(logo.make_shape(q, k), w.ratio, q.device)
+    out, sel, cu_sel = logo.forward(q, k, v, g, w.W, w.ratio, ws=ws)
+    logo.check(ws)
+    ref = oracle.forward(w.q, w.k, w.v, w.g, w.W, w.ratio, want_branches=True)
+    assert sel_lists(sel, cu_sel) == oracle_sel_lists(w)
+    loc = logo.local_attn(q, k, v, w.W, ws)
+    logo.check(ws)
+    for got, r, what in ((loc, ref["local"], "local"), (out, ref["out"], "merged")):
+        bound = MAX_ABS * max(1.0, r.abs().max().item() / 4.0)
+        close(got, r, what, max_abs=bound)
+
+
+def test_forward_deterministic_under_max_growth():
+    """Bitwise-identical outputs across repeated runs (plain and training forward) on a
+    16K-token workload whose key norms ramp x1 -> x9, so rows rescale their running
+    softmax state on many key tiles after the first (the path where the two P parts
+    and the O rescale must not overlap)."""
+    L = 16384
+    w = workloads.make(1, 8, 2, L, 128, 4096, 0.2, seed=9, qkv_scale=1.0, name="ramp16k")
+    f = 1.0 + 8.0 * torch.arange(L, dtype=torch.float32) / L
+    w.k = (w.k.float() * f[None, None, :, None]).bfloat16()
+    q, k, v, g, cu = to_dev(w)
+    first, _, _ = logo.forward(q, k, v, g, w.W, w.ratio)
+    for _ in range(3):
+        again, _, _ = logo.forward(q, k, v, g, w.W, w.ratio)
+        assert torch.equal(again, first), "forward is not deterministic"
+    tr, _ = logo.forward_train(q, k, v, g, w.W, w.ratio)
+    assert torch.equal(tr, first), "training forward differs from the plain forward"
 
 
 def test_forward_is_deterministic():

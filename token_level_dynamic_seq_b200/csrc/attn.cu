@@ -36,7 +36,10 @@
 //   PV_i(j), S_i(j+1).  S_i(j+1) overwrites the TMEM columns of P_i(j) only
 //   after PV_i(j) has read them, because tcgen05 MMAs from one thread execute
 //   in issue order; and the commit that signals S_i(j+1) also covers
-//   PV_i(j), so a softmax warpgroup may rescale O_i as soon as it sees S_i(j+1).
+//   PV_i(j), so O_i may be rescaled as soon as S_i(j+1) is seen.  P_i(j) is
+//   published in two parts (one per half-row warpgroup) and the MMAs of the
+//   first part write all of O_i, so only the first half's warpgroup rescales
+//   O_i (every column), before it publishes its part.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -63,12 +66,12 @@ static_assert(kPParts == 2, "P is published in two parts, one per half-row warpg
 #ifndef LOGO_POLY_EVERY
 #define LOGO_POLY_EVERY 0
 #endif
-// Every kPolyEvery-th exponential of a row uses exp2_poly (FMA pipe) instead
-// of the MUFU unit; 0 keeps them all on MUFU.
+// Every kPolyEvery-th pair of exponentials of a row uses exp2_poly2 (FMA pipe)
+// instead of the MUFU unit; 0 keeps them all on MUFU.
 constexpr int kPolyEvery = LOGO_POLY_EVERY;
-__device__ __forceinline__ constexpr bool use_poly(int col)
+__device__ __forceinline__ constexpr bool use_poly(int pair)
 {
-    return kPolyEvery > 0 && (col % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
+    return kPolyEvery > 0 && (pair % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
 }
 
 template <int D>
@@ -394,7 +397,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const uint32_t tS = tmem + lane_off + Geo::kTmemS + 128 * wg + 64 * half;  // this half's S
         const uint32_t tP = tmem + lane_off + Geo::kTmemS + 128 * wg + 32 * half;  // this half's P
-        const uint32_t tO = tmem + lane_off + Geo::kTmemO + D * wg + (D / 2) * half;
+        const uint32_t tO_row = tmem + lane_off + Geo::kTmemO + D * wg;  // all D columns of O for this row
+        const uint32_t tO = tO_row + (D / 2) * half;                       // this half's D/2 columns
         float* xch = xchg + (wg * 2) * 128;       // [2][128]: one value per row from each half
         uint64_t* pair = &pair_bar[wg];
         // Per-tile fields picked with selects (no dynamic indexing into Work).
@@ -480,37 +484,53 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 l_run *= alpha;
             }
             const float mref = (m_run == -INFINITY) ? 0.f : m_run * sl2;
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};
             __syncwarp();
+            // Paired fp32 instructions for the scaling and the row sums.
+            const uint64_t sl2x2 = f2_pack(sl2, sl2), nmref2 = f2_pack(-mref, -mref);
+            uint64_t ls2[2] = {0ull, 0ull};
             #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t pk[16];
                 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                     const int col = 64 * half + c * 32 + e;
-                    const float x0 = fmaf(__uint_as_float(sr[c][e]), sl2, -mref);
-                    const float x1 = fmaf(__uint_as_float(sr[c][e + 1]), sl2, -mref);
-                    // A share of the exponentials may run on the FMA pipe to unload the MUFU unit.
-                    const float p0 = use_poly(col) ? exp2_poly(x0) : fast_exp2(x0);
-                    const float p1 = use_poly(col + 1) ? exp2_poly(x1) : fast_exp2(x1);
-                    ls[(e >> 1) & 3] += p0 + p1;
+                    float x0, x1, p0, p1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), sl2x2, nmref2),
+                              x0, x1);
+                    // A share of the pairs may run on the FMA pipe to unload the MUFU unit.
+                    if (use_poly(col / 2)) {
+                        exp2_poly2(x0, x1, p0, p1);
+                    } else {
+                        p0 = fast_exp2(x0);
+                        p1 = fast_exp2(x1);
+                    }
+                    ls2[(e >> 1) & 1] = f2_add(ls2[(e >> 1) & 1], f2_pack(p0, p1));
                     pk[e / 2] = pack_bf16x2(p0, p1);
                 }
                 tmem_st16(tP + c * 16, pk);
             }
-            l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-            // Rare: the row maximum grew past the threshold, so rescale this half's
-            // columns of O (PV of tile j-1 is complete: see header) before its PV.
+            {
+                const uint64_t lsum = f2_add(ls2[0], ls2[1]);
+                float l0, l1;
+                f2_unpack(lsum, l0, l1);
+                l_run += l0 + l1;
+            }
+            // Rare: the row maximum grew past the threshold, so O must be rescaled
+            // before any PV of this tile (PV of tile j-1 is complete: see header).
+            // The first half rescales all D columns of the row: the first P part's
+            // MMAs (issued as soon as this half has arrived) write every column of
+            // O, so the second half must not touch O while they may run.  Both
+            // halves took the same decision and hold the same alpha.
             const bool any = __any_sync(0xffffffffu, need);  // also reconverges the warp
-            if (any && j > 0) {
+            if (any && j > 0 && half == 0) {
                 #pragma unroll 1
-                for (int c = 0; c < D / 64; ++c) {
+                for (int c = 0; c < D / 32; ++c) {
                     uint32_t orr[32];
-                    tmem_ld32(tO + c * 32, orr);
+                    tmem_ld32(tO_row + c * 32, orr);
                     tmem_wait_ld(orr);
                     #pragma unroll
                     for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-                    tmem_st32(tO + c * 32, orr);
+                    tmem_st32(tO_row + c * 32, orr);
                 }
             }
             tmem_wait_st();

@@ -474,22 +474,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             const int hi = pos - kbase;
             const int lo = (MODE == kModeLocal) ? pos - W + 1 - kbase : INT_MIN;
             // P = exp2(S * scale * log2(e) - lse); the mask as selects behind a uniform test.
+            // Paired fp32 instructions: x = S * sl2 - lse for two columns at once.
+            const uint64_t sl2x2 = f2_pack(sl2, sl2), nlse2 = f2_pack(-lse2, -lse2);
             if (need_mask) {
                 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
+                    for (int e = 0; e < 32; e += 2) {
                         const int col = c * 32 + e;
-                        const float x = fmaf(__uint_as_float(sr[c][e]), sl2, -lse2);
-                        sr[c][e] = __float_as_uint(fast_exp2((col <= hi) & (col >= lo) ? x : -INFINITY));
+                        float x0, x1;
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), sl2x2, nlse2),
+                                  x0, x1);
+                        sr[c][e] = __float_as_uint(fast_exp2((col <= hi) & (col >= lo) ? x0 : -INFINITY));
+                        sr[c][e + 1] = __float_as_uint(fast_exp2((col + 1 <= hi) & (col + 1 >= lo) ? x1 : -INFINITY));
                     }
                 }
             } else {
                 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        sr[c][e] = __float_as_uint(fast_exp2(fmaf(__uint_as_float(sr[c][e]), sl2, -lse2)));
+                    for (int e = 0; e < 32; e += 2) {
+                        float x0, x1;
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), sl2x2, nlse2),
+                                  x0, x1);
+                        sr[c][e] = __float_as_uint(fast_exp2(x0));
+                        sr[c][e + 1] = __float_as_uint(fast_exp2(x1));
+                    }
                 }
             }
             ok = __all_sync(0xffffffffu, mbar_wait(dp_full, j & 1, abort_flag, p.status, limit));
@@ -502,11 +512,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                 tmem_ld32(tD + 32 * c, dp);
                 tmem_wait_ld(dp);
                 uint32_t pk[16];
+                const uint64_t ndsum2 = f2_pack(-dsum, -dsum);
                 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    const float p0 = __uint_as_float(sr[c][e]), p1 = __uint_as_float(sr[c][e + 1]);
-                    const float d0 = p0 * (__uint_as_float(dp[e]) - dsum);
-                    const float d1 = p1 * (__uint_as_float(dp[e + 1]) - dsum);
+                    // dS = P * (dP - D), two columns per instruction
+                    const uint64_t p2 = f2_pack(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+                    const uint64_t dp2 = f2_pack(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1]));
+                    float d0, d1;
+                    f2_unpack(f2_mul(p2, f2_add(dp2, ndsum2)), d0, d1);
                     pk[e / 2] = pack_bf16x2(d0, d1);
                 }
                 // Columns 16c .. 16c+15 of this half: dP there has been read (chunk 0 above).
@@ -777,19 +790,19 @@ __global__ void __launch_bounds__(kKvThreads) bwd_dkdv_kernel(const __grid_const
             for (int u = 0; u < 4; ++u) {
                 const int c = lane * 4 + u;
                 qp[u] = 0;
-                l2[u] = INFINITY;
+                l2[u] = -INFINITY;  // minus the query's lse (a column past the end gets P = 0)
                 dd[u] = 0.f;
                 if (local) {
                     qp[u] = q0 + c;
                     if (qp[u] < len) {
                         const size_t idx = ((size_t)(b * p.Hq + h)) * p.L + s0 + qp[u];
-                        l2[u] = __ldg(p.lse + idx);
+                        l2[u] = -__ldg(p.lse + idx);
                         dd[u] = __ldg(p.dl + idx);
                     }
                 } else if (q0 + c < k_sel) {
                     qp[u] = __ldg(p.sel_idx + sel_base + q0 + c);
                     const size_t idx = (size_t)h * p.sel_stride + sel_base + q0 + c;
-                    l2[u] = __ldg(p.lse_s + idx);
+                    l2[u] = -__ldg(p.lse_s + idx);
                     dd[u] = __ldg(p.ds_sel + idx);
                 }
             }
@@ -886,7 +899,7 @@ __global__ void __launch_bounds__(kKvThreads) bwd_dkdv_kernel(const __grid_const
             const int m = n % per_head;
             const bool local = m < nl;
             const int* cpos = scol + cs * 384 + 64 * half;
-            const float* clse = reinterpret_cast<const float*>(scol + cs * 384 + 128 + 64 * half);
+            const float* cnlse = reinterpret_cast<const float*>(scol + cs * 384 + 128 + 64 * half);
             const float* cdd = reinterpret_cast<const float*>(scol + cs * 384 + 256 + 64 * half);
             ok = __all_sync(0xffffffffu, mbar_wait(&col_full[cs], (n / kColStages) & 1, abort_flag, p.status, limit));
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full, n & 1, abort_flag, p.status, limit));
@@ -908,12 +921,12 @@ __global__ void __launch_bounds__(kKvThreads) bwd_dkdv_kernel(const __grid_const
             const int wl = local ? W : INT_MAX;  // a query more than wl - 1 past the key is out
             // P^T = exp2(S^T * scale * log2(e) - lse(query)); the mask, where the tile needs it,
             // as selects (a per-element branch here costs more than the exponentials).
+            const uint64_t sl2x2 = f2_pack(sl2, sl2);
             auto p_chunk = [&](int c, auto masked) {
                 #pragma unroll
                 for (int e4 = 0; e4 < 32; e4 += 4) {
                     const int col = c * 32 + e4;
-                    const float4 l4 = *reinterpret_cast<const float4*>(clse + col);
-                    const float la[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float4 nl4 = *reinterpret_cast<const float4*>(cnlse + col);  // -lse per column
                     int qa[4] = {0, 0, 0, 0};
                     if (decltype(masked)::value) {
                         const int4 q4 = *reinterpret_cast<const int4*>(cpos + col);
@@ -922,14 +935,21 @@ __global__ void __launch_bounds__(kKvThreads) bwd_dkdv_kernel(const __grid_const
                         qa[2] = q4.z;
                         qa[3] = q4.w;
                     }
+                    // x = S^T * sl2 - lse, two columns per paired instruction
+                    float x[4];
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c][e4]), __uint_as_float(sr[c][e4 + 1])), sl2x2,
+                                     f2_pack(nl4.x, nl4.y)),
+                              x[0], x[1]);
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c][e4 + 2]), __uint_as_float(sr[c][e4 + 3])), sl2x2,
+                                     f2_pack(nl4.z, nl4.w)),
+                              x[2], x[3]);
                     #pragma unroll
                     for (int t = 0; t < 4; ++t) {
-                        float x = fmaf(__uint_as_float(sr[c][e4 + t]), sl2, -la[t]);
                         if (decltype(masked)::value) {
                             const int dq = qa[t] - kp;
-                            x = (dq >= 0) & (dq < wl) ? x : -INFINITY;
+                            x[t] = (dq >= 0) & (dq < wl) ? x[t] : -INFINITY;
                         }
-                        sr[c][e4 + t] = __float_as_uint(fast_exp2(x));
+                        sr[c][e4 + t] = __float_as_uint(fast_exp2(x[t]));
                     }
                 }
             };
@@ -955,11 +975,16 @@ __global__ void __launch_bounds__(kKvThreads) bwd_dkdv_kernel(const __grid_const
                 #pragma unroll
                 for (int e4 = 0; e4 < 32; e4 += 4) {
                     const float4 d4 = *reinterpret_cast<const float4*>(cdd + c * 32 + e4);
-                    const float da[4] = {d4.x, d4.y, d4.z, d4.w};
+                    // dS^T = P^T * (dP^T - D), two columns per paired instruction
                     float ds[4];
-                    #pragma unroll
-                    for (int t = 0; t < 4; ++t)
-                        ds[t] = __uint_as_float(sr[c][e4 + t]) * (__uint_as_float(dp[e4 + t]) - da[t]);
+                    f2_unpack(f2_mul(f2_pack(__uint_as_float(sr[c][e4]), __uint_as_float(sr[c][e4 + 1])),
+                                     f2_sub(f2_pack(__uint_as_float(dp[e4]), __uint_as_float(dp[e4 + 1])),
+                                            f2_pack(d4.x, d4.y))),
+                              ds[0], ds[1]);
+                    f2_unpack(f2_mul(f2_pack(__uint_as_float(sr[c][e4 + 2]), __uint_as_float(sr[c][e4 + 3])),
+                                     f2_sub(f2_pack(__uint_as_float(dp[e4 + 2]), __uint_as_float(dp[e4 + 3])),
+                                            f2_pack(d4.z, d4.w))),
+                              ds[2], ds[3]);
                     pk[e4 / 2] = pack_bf16x2(ds[0], ds[1]);
                     pk[e4 / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
                     pp[e4 / 2] = pack_bf16x2(__uint_as_float(sr[c][e4]), __uint_as_float(sr[c][e4 + 1]));

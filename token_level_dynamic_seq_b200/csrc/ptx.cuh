@@ -290,6 +290,68 @@ LOGO_DEVICE_INLINE float exp2_poly(float x)
     return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// Paired fp32 arithmetic (one instruction for two lanes of a 64-bit register
+// pair; sm_100 and later).  f2 values hold {lo, hi}.
+LOGO_DEVICE_INLINE uint64_t f2_pack(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+LOGO_DEVICE_INLINE void f2_unpack(uint64_t v, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+LOGO_DEVICE_INLINE uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+LOGO_DEVICE_INLINE uint64_t f2_add(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+LOGO_DEVICE_INLINE uint64_t f2_sub(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+LOGO_DEVICE_INLINE uint64_t f2_mul(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// exp2_poly on a pair, with the additions and the polynomial in paired
+// instructions: the same arithmetic and result bits as exp2_poly per lane.
+LOGO_DEVICE_INLINE void exp2_poly2(float x0, float x1, float& y0, float& y1)
+{
+    const uint64_t x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+    const uint64_t t = f2_add(x, f2_pack(12582912.0f, 12582912.0f));
+    const uint64_t n = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
+    const uint64_t f = f2_sub(x, n);
+    const float c3 = __uint_as_float(0x3d61fbb0u), c2 = __uint_as_float(0x3e786f0du);
+    const float c1 = __uint_as_float(0x3f31798du), c0 = __uint_as_float(0x3f7ffb49u);
+    uint64_t p = f2_fma(f2_pack(c3, c3), f, f2_pack(c2, c2));
+    p = f2_fma(p, f, f2_pack(c1, c1));
+    p = f2_fma(p, f, f2_pack(c0, c0));
+    float p0, p1, t0, t1;
+    f2_unpack(p, p0, p1);
+    f2_unpack(t, t0, t1);
+    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 LOGO_DEVICE_INLINE uint32_t pack_bf16x2(float lo, float hi)
 {
     uint32_t r;
