@@ -70,6 +70,15 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
+def decode_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("decode.cu", "ptx.cuh", "kernels.cuh"):
+        with open(os.path.join(ROOT, "token_level_dynamic_seq_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def traffic_record():
     """DRAM bytes per launch from the committed ncu summary, if taken on the current kernel source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -79,6 +88,18 @@ def traffic_record():
     except Exception:
         return {}
     return rec if rec.get("source_hash") == kernel_source_hash() else {}
+
+
+def decode_traffic_record():
+    """DRAM bytes of one decode step (both kernels) from the committed ncu summary, if taken on
+    the current decode source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get("decode", {})
+    except Exception:
+        return {}
+    return rec if rec.get("source_hash") == decode_source_hash() else {}
 
 
 class ClockSampler:
@@ -268,7 +289,8 @@ def run_decode(args, rank, world):
                    "ratio": ratio, "selected": n_sel,
                    "l2": f"caches ({kc.numel() * 4 / 1e9:.1f} GB) larger than L2"},
         "roofline": {"kernel": "decode_partial_kernel + decode_combine_kernel", "bound": "hbm",
-                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": decode_traffic_record().get("bytes_per_step") if B == 64 else None,
                      "peak_source": f"{peak_src} HBM copy bandwidth"},
         "gpu_launches": 2 * args.steps, "clocks": clocks,
     }

@@ -128,21 +128,26 @@ EncodeTiledFn encode_fn(logo_status& st)
     return fn;
 }
 
-// 3-D bf16 view [slabs][rows][d] with a box of 64 x 128 x 1 and the 128B swizzle.
-logo_status make_map(CUtensorMap* map, const void* base, int d, int rows, int slabs)
+// 3-D bf16 view [slabs][rows][d] with a box of 64 x box_rows x 1 and the 128B swizzle.
+logo_status make_map_box(CUtensorMap* map, const void* base, int d, int rows, int slabs, int box_rows)
 {
     logo_status st;
     EncodeTiledFn fn = encode_fn(st);
     if (!fn) return st;
     cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)(rows > 0 ? rows : 1), (cuuint64_t)slabs};
     cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * (cuuint64_t)(rows > 0 ? rows : 1)};
-    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(LOGO_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return LOGO_OK;
+}
+
+logo_status make_map(CUtensorMap* map, const void* base, int d, int rows, int slabs)
+{
+    return make_map_box(map, base, d, rows, slabs, 128);
 }
 
 void base_params(AttnParams& p, const Geo& g, const void* q, const void* k, const void* v, void* out,
@@ -604,6 +609,7 @@ logo_status logo_decode(const logo_bf16* q, const logo_bf16* k_cache, const logo
     if (selected && (reinterpret_cast<uintptr_t>(selected) & 3u))
         return fail(LOGO_ERR_INVALID_ARG, "selected is not 4-byte aligned");
     logo::DecodeParams p;
+    memset(&p, 0, sizeof p);
     p.q = reinterpret_cast<const uint16_t*>(q);
     p.k = reinterpret_cast<const uint16_t*>(k_cache);
     p.v = reinterpret_cast<const uint16_t*>(v_cache);
@@ -624,6 +630,12 @@ logo_status logo_decode(const logo_bf16* q, const logo_bf16* k_cache, const logo
     p.chunk = logo::kDecChunk;
     p.nchunks = g.L > 0 ? (g.L + logo::kDecChunk - 1) / logo::kDecChunk : 1;
     p.scale_log2 = sl2;
+    p.timeout_ns = 1000000000ull;  // 1 s per wait: far above any legitimate stall
+    if (g.L > 0) {
+        if ((st = make_map_box(&p.tm_k, k_cache, g.d, g.L, g.B * g.Hkv, logo::kDecBlock)) != LOGO_OK ||
+            (st = make_map_box(&p.tm_v, v_cache, g.d, g.L, g.B * g.Hkv, logo::kDecBlock)) != LOGO_OK)
+            return st;
+    }
     cudaError_t e = logo::launch_decode(p, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? LOGO_OK : cuda_fail(e, "decode launch");
 }

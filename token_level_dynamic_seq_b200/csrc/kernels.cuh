@@ -85,8 +85,10 @@ cudaError_t launch_threshold_update(const float* gate, const int32_t* cu_seqlens
                                     double ratio, float beta, float* tau, float* target_out, cudaStream_t stream);
 
 // Decode step (decode.cu).
-constexpr int kDecChunk = 512;  // cache positions per partial CTA
+constexpr int kDecChunk = 512;  // cache positions per partial state
+constexpr int kDecBlock = 16;   // cache positions per staged key/value block
 struct DecodeParams {
+    CUtensorMap tm_k, tm_v;     // caches as [B*Hkv][Lmax][d], box 64 x kDecBlock x 1, 128B swizzle
     const uint16_t *q, *k, *v;  // q [B, Hq, d]; caches [B, Hkv, Lmax, d]
     const int32_t* cache_len;   // [B]: the new token sits at cache_len - 1
     const float* gate;          // [B]
@@ -97,6 +99,7 @@ struct DecodeParams {
     uint32_t* status;           // workspace status word
     int B, Hq, Hkv, G, Lmax, d, W, chunk, nchunks;
     float scale_log2;
+    unsigned long long timeout_ns;  // bound of every barrier wait
 };
 size_t decode_partials_bytes(int B, int Hkv, int G, int Lmax, int d);
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
