@@ -31,12 +31,13 @@
  *
  * Conventions shared by every entry point:
  *   - Ownership: the caller owns every buffer and the stream.  The library
- *     allocates no memory and never synchronises, except logo_check.  Every
- *     call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
- *     stream).
+ *     allocates no memory and never synchronises, except logo_check
+ *     (logo_forward_host creates, once per device, two internal streams and a
+ *     few events for its copy pipeline).  Every call is asynchronous on
+ *     `stream` (a cudaStream_t; NULL = legacy default stream).
  *   - Device pointers: q, k, v, out, gate, sel_idx, cu_sel, cu_seqlens and ws
  *     are device (HBM) pointers on the current device, 16-byte aligned,
- *     contiguous in the stated layout.
+ *     contiguous in the stated layout (logo_forward_host takes host buffers).
  *   - Element types: q, k, v, out are bf16 (passed as raw 16-bit patterns);
  *     gate is fp32; indices are int32.
  *   - Errors: argument problems are reported synchronously as a logo_status
@@ -217,6 +218,38 @@ LOGO_API logo_status logo_forward(const logo_bf16 *q, const logo_bf16 *k, const 
                          const logo_shape *shape, int window, double ratio, float scale, logo_bf16 *out,
                          int32_t *sel_idx, int32_t *cu_sel, void *ws, size_t ws_bytes,
                          logo_stream_t stream);
+
+/*
+ * The same forward pass with the tensors in HOST memory (the call a user with
+ * data on the host makes).  Computes exactly what logo_forward computes, with
+ * the same kernels, one key/value-head group at a time: the gate is copied in
+ * and the selection made once; then, per group, its Q, K and V rows are copied
+ * into a device slot, the local and global kernels run on them, and its output
+ * rows are copied back, the copies of neighbouring groups overlapping the
+ * kernels (three rotating slots, two internal streams joined back to `stream`).
+ *   q, k, v, gate, out: host buffers with logo_forward's layouts (page-locked
+ *     memory lets the copies run asynchronously; pageable memory still works).
+ *   shape: as for logo_forward, except that shape->cu_seqlens, when given, is a
+ *     HOST array of nseq + 1 offsets.
+ *   sel_idx, cu_sel: host buffers receiving the selection (nseq * k_max int32
+ *     with k_max = logo_num_selected(ratio, max_seqlen), lists back to back as in
+ *     logo_select, and nseq + 1 offsets), or NULL.
+ *   dev_buf: a device arena of logo_forward_host_buffer_size(shape, ratio)
+ *     bytes, 16-byte aligned, owned by the caller; its first bytes are the
+ *     workspace: initialise it once with logo_workspace_init(dev_buf, ...) and
+ *     read the device status with logo_check(dev_buf, stream).
+ * Asynchronous: returns once everything is queued; `stream` completes after the
+ * last output copy, so synchronise it before reading out/sel_idx/cu_sel or
+ * reusing the inputs.  Calls are serialised by an internal lock.  Errors: the
+ * argument errors of logo_forward, LOGO_ERR_WORKSPACE for a missing or small
+ * arena, LOGO_ERR_CUDA when a copy, stream or event call fails (the stream is
+ * then left partly queued: synchronise the device before reuse).
+ */
+LOGO_API size_t logo_forward_host_buffer_size(const logo_shape *shape, double ratio);
+LOGO_API logo_status logo_forward_host(const logo_bf16 *q, const logo_bf16 *k, const logo_bf16 *v,
+                                       const float *gate, const logo_shape *shape, int window, double ratio,
+                                       float scale, logo_bf16 *out, int32_t *sel_idx, int32_t *cu_sel,
+                                       void *dev_buf, size_t dev_buf_bytes, logo_stream_t stream);
 
 /*
  * The same computation as logo_global_attn_sparse (same arguments, same

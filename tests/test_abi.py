@@ -32,7 +32,7 @@ def declared_symbols():
 def test_library_exports_every_declared_symbol():
     lib = logo.load_library()
     names = declared_symbols()
-    assert len(names) == 19, names
+    assert len(names) == 21, names
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(logo.EXPORTED)
@@ -162,3 +162,24 @@ def test_training_entry_points_reject():
     assert bw(ws_bytes=need - 1) == 3
     assert bw(dout=None) == 1
     assert lib.logo_last_error().decode() != ""
+
+
+def test_host_forward_entry_rejects():
+    """The host-buffer forward validates its arguments before touching the device."""
+    lib = logo.load_library()
+    sh = shape()
+    by = ctypes.byref(sh)
+    need = lib.logo_forward_host_buffer_size(by, 0.2)
+    # arena = workspace + gate + selection + three slots of one kv-head group's Q, O, K, V
+    assert need > 3 * 2 * (sh.B * (sh.Hq // sh.Hkv) * sh.L * sh.d * 2)
+    assert lib.logo_forward_host_buffer_size(ctypes.byref(shape(d=96)), 0.2) == 0
+    assert lib.logo_forward_host_buffer_size(by, 1.5) == 0
+    fh = lambda **kw: lib.logo_forward_host(
+        FAKE, FAKE, FAKE, kw.get("gate", FAKE), kw.get("by", by), kw.get("window", 8), kw.get("ratio", 0.2), 0.0,
+        FAKE2, None, None, kw.get("buf", FAKE), kw.get("nbytes", need), None)
+    assert fh(window=0) == 1
+    assert fh(ratio=-0.5) == 1
+    assert fh(by=ctypes.byref(shape(d=96))) == 2
+    assert fh(buf=None) == 3
+    assert fh(nbytes=need - 1) == 3
+    assert fh(gate=None) == 1

@@ -187,6 +187,34 @@ def test_forward_deterministic_under_max_growth():
     assert torch.equal(tr, first), "training forward differs from the plain forward"
 
 
+HOST_CASES = [
+    # name, B, Hq, Hkv, L, d, W, ratio, seqlens
+    ("host gqa4 b2", 2, 8, 2, 700, 128, 256, 0.2, None),
+    ("host 4 kv heads (slot reuse)", 1, 8, 4, 1000, 128, 300, 0.2, None),
+    ("host g3 d64", 1, 3, 1, 513, 64, 200, 0.3, None),
+    ("host varlen", 1, 4, 2, 0, 128, 100, 0.25, [1, 130, 0, 700, 255]),
+]
+
+
+@pytest.mark.parametrize("case", HOST_CASES, ids=[c[0] for c in HOST_CASES])
+def test_forward_host_matches_device(case):
+    """logo_forward_host (host buffers, per kv-head-group copy pipeline) gives the same
+    bits as logo_forward on device buffers, and the same selection."""
+    w = small_workload(case)
+    ml = max_len(w)
+    pinned = [x.contiguous().pin_memory() for x in (w.q, w.k, w.v, w.g)]
+    cu_host = None if w.cu_seqlens is None else w.cu_seqlens.clone()
+    out_h, sel_h, cu_sel_h = logo.forward_host(*pinned, w.W, w.ratio, cu_seqlens=cu_host, max_seqlen=ml)
+    torch.cuda.synchronize()
+    q, k, v, g, cu = to_dev(w)
+    out_d, sel_d, cu_sel_d = logo.forward(q, k, v, g, w.W, w.ratio, cu_seqlens=cu, max_seqlen=ml)
+    torch.cuda.synchronize()
+    assert cu_sel_h.tolist() == cu_sel_d.cpu().tolist()
+    n = int(cu_sel_h[-1])
+    assert sel_h[:n].tolist() == sel_d[:n].cpu().tolist()
+    assert torch.equal(out_h, out_d.cpu()), "host-buffer forward differs from the device forward"
+
+
 def test_forward_is_deterministic():
     w = small_workload(SMALL[7], seed=3)
     q, k, v, g, cu = to_dev(w)

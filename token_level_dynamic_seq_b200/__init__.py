@@ -36,7 +36,7 @@ EXPORTED = ("logo_num_selected", "logo_workspace_size", "logo_workspace_init", "
             "logo_selftest_timeout", "logo_status_string", "logo_last_error",
             "logo_global_attn_sparse_noalloc", "logo_select_threshold", "logo_threshold_update",
             "logo_decode_workspace_size", "logo_decode", "logo_forward_train", "logo_backward_workspace_size",
-            "logo_backward")
+            "logo_backward", "logo_forward_host_buffer_size", "logo_forward_host")
 
 
 class LogoError(RuntimeError):
@@ -89,6 +89,8 @@ def load_library(path: str | None = None):
             "logo_forward_train": ([vp, vp, vp, vp, sp, i32, dbl, flt, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp],
                                    i32),
             "logo_backward_workspace_size": ([sp, i32], sz),
+            "logo_forward_host_buffer_size": ([sp, dbl], sz),
+            "logo_forward_host": ([vp, vp, vp, vp, sp, i32, dbl, flt, vp, vp, vp, vp, sz, vp], i32),
             "logo_backward": ([vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sp, i32, flt, vp, vp, vp,
                                vp, vp, sz, vp], i32),
         }
@@ -278,6 +280,59 @@ def forward(q, k, v, gate, window: int, ratio: float, ws: torch.Tensor | None = 
     _raise(load_library().logo_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(gate), ctypes.byref(shape), int(window),
                                        float(ratio), float(scale), _ptr(out), _ptr(sel_idx), _ptr(cu_sel),
                                        _ptr(ws), ws.numel(), _stream(stream)))
+    return out, sel_idx, cu_sel
+
+
+def _host_bits(x: torch.Tensor) -> torch.Tensor:
+    if x.dtype != torch.bfloat16:
+        raise TypeError(f"expected bf16, got {x.dtype}")
+    if x.is_cuda:
+        raise ValueError("expected a host tensor")
+    if not x.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return x
+
+
+def host_buffer(shape: Shape, ratio: float, device, stream=None) -> torch.Tensor:
+    """Device arena of :func:`forward_host` (its first bytes are the workspace, initialised here)."""
+    lib = load_library()
+    n = lib.logo_forward_host_buffer_size(ctypes.byref(shape), float(ratio))
+    if n == 0:
+        _raise(1)
+    buf = torch.empty(n, dtype=torch.uint8, device=device)
+    _raise(lib.logo_workspace_init(_ptr(buf), buf.numel(), _stream(stream)))
+    return buf
+
+
+def forward_host(q, k, v, gate, window: int, ratio: float, buf: torch.Tensor | None = None, device=None,
+                 scale: float = 0.0, cu_seqlens=None, max_seqlen=None, out=None, sel_idx=None, cu_sel=None,
+                 stream=None):
+    """The whole forward pass on HOST tensors (page-locked for asynchronous copies).
+
+    The library copies the inputs in and the output out, one key/value-head group
+    at a time, overlapping the copies with the kernels.  ``cu_seqlens`` (packed
+    layout) is a host int32 tensor here.  Returns host tensors (out, sel_idx,
+    cu_sel) once the work is queued on ``stream``: synchronise the stream before
+    reading them.  ``buf`` is the device arena (:func:`host_buffer`)."""
+    q, k, v = _host_bits(q), _host_bits(k), _host_bits(v)
+    if gate.is_cuda or gate.dtype != torch.float32:
+        raise ValueError("gate must be a host fp32 tensor")
+    shape = make_shape(q, k, cu_seqlens, max_seqlen)
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    if buf is None:
+        buf = host_buffer(shape, ratio, device, stream)
+    nseq = shape.nseq if cu_seqlens is not None else shape.B
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    if sel_idx is None:
+        sel_idx = torch.empty(max(1, nseq * num_selected(ratio, shape.max_seqlen)), dtype=torch.int32,
+                              pin_memory=True)
+    if cu_sel is None:
+        cu_sel = torch.empty(nseq + 1, dtype=torch.int32, pin_memory=True)
+    _raise(load_library().logo_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(gate), ctypes.byref(shape),
+                                            int(window), float(ratio), float(scale), _ptr(out), _ptr(sel_idx),
+                                            _ptr(cu_sel), _ptr(buf), buf.numel(), _stream(stream)))
     return out, sel_idx, cu_sel
 
 

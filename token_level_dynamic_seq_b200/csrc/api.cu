@@ -264,6 +264,79 @@ BwdWs bwd_layout(const Geo& g, int cap)
     return w;
 }
 
+// ---------------------------------------------------------------- host-buffer forward
+//
+// Layout of the device arena of logo_forward_host (every part 256-byte aligned):
+//   workspace (header + per-sequence counts) | gate | cu_seqlens (packed only) |
+//   selection lists | cu_sel | kHostSlots x (Q, K, V, O of one kv-head group).
+constexpr int kHostSlots = 3;
+
+struct HostArena {
+    size_t ws, gate, cu, sel, cu_sel, slot0, slot_bytes, q_bytes, kv_bytes, total, ws_bytes;
+    int sel_cap;
+};
+
+size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+HostArena host_arena(const Geo& g, double ratio)
+{
+    HostArena a;
+    const int max_sel = (int)logo::budget_count(ratio, g.max_len);
+    a.sel_cap = g.nseq * max_sel;
+    a.ws_bytes = kWsHeaderBytes + counts_bytes(g.nseq);
+    a.ws = 0;
+    a.gate = up256(a.ws_bytes);
+    a.cu = a.gate + up256((size_t)g.B * g.L * sizeof(float));
+    a.sel = a.cu + (g.cu ? up256((size_t)(g.nseq + 1) * 4) : 0);
+    a.cu_sel = a.sel + up256((size_t)(a.sel_cap > 0 ? a.sel_cap : 1) * 4);
+    a.slot0 = a.cu_sel + up256((size_t)(g.nseq + 1) * 4);
+    a.q_bytes = (size_t)g.B * g.G * g.L * g.d * 2;
+    a.kv_bytes = (size_t)g.B * g.L * g.d * 2;
+    a.slot_bytes = up256(a.q_bytes) * 2 + up256(a.kv_bytes) * 2;  // Q, O, K, V
+    const int slots = g.Hkv < kHostSlots ? g.Hkv : kHostSlots;
+    a.total = a.slot0 + (size_t)slots * a.slot_bytes;
+    return a;
+}
+
+// Streams and events of the copy pipeline, one set per device, created on first use.
+struct HostPipe {
+    bool ready = false;
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t start, inputs, sel_done, h2d, comp, done, d2h[kHostSlots];
+};
+std::mutex g_host_mu;
+HostPipe g_host_pipes[64];
+
+cudaError_t host_pipe(int dev, HostPipe*& hp)
+{
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    hp = &g_host_pipes[dev];
+    if (hp->ready) return cudaSuccess;
+    cudaError_t e;
+    if ((e = cudaStreamCreateWithFlags(&hp->in, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithFlags(&hp->out, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    cudaEvent_t* evs[] = {&hp->start, &hp->inputs, &hp->sel_done, &hp->h2d, &hp->comp, &hp->done};
+    for (cudaEvent_t* ev : evs)
+        if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+    for (int i = 0; i < kHostSlots; ++i)
+        if ((e = cudaEventCreateWithFlags(&hp->d2h[i], cudaEventDisableTiming)) != cudaSuccess) return e;
+    hp->ready = true;
+    return cudaSuccess;
+}
+
+// `rows` copies of `row_bytes` each, source and destination rows `src_pitch` /
+// `dst_pitch` bytes apart (one cudaMemcpyAsync per row).
+cudaError_t copy_rows(void* dst, size_t dst_pitch, const void* src, size_t src_pitch, size_t row_bytes, int rows,
+                      cudaMemcpyKind kind, cudaStream_t s)
+{
+    for (int r = 0; r < rows; ++r) {
+        cudaError_t e = cudaMemcpyAsync(static_cast<uint8_t*>(dst) + r * dst_pitch,
+                                        static_cast<const uint8_t*>(src) + r * src_pitch, row_bytes, kind, s);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
 }  // namespace
 
 extern "C" {
@@ -668,6 +741,111 @@ logo_status logo_selftest_timeout(void* ws, size_t ws_bytes, unsigned limit_us, 
     cudaError_t e = logo::launch_timeout_probe(static_cast<uint32_t*>(ws), 1000ull * limit_us,
                                                static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? LOGO_OK : cuda_fail(e, "timeout probe launch");
+}
+
+size_t logo_forward_host_buffer_size(const logo_shape* shape, double ratio)
+{
+    Geo g;
+    if (check_shape(shape, g) != LOGO_OK || check_ratio(ratio) != LOGO_OK) return 0;
+    return host_arena(g, ratio).total;
+}
+
+logo_status logo_forward_host(const logo_bf16* q, const logo_bf16* k, const logo_bf16* v, const float* gate,
+                              const logo_shape* shape, int window, double ratio, float scale, logo_bf16* out,
+                              int32_t* sel_idx, int32_t* cu_sel, void* dev_buf, size_t dev_buf_bytes,
+                              logo_stream_t stream)
+{
+    Geo g;
+    logo_status st;
+    float sl2;
+    if ((st = check_shape(shape, g)) != LOGO_OK) return st;
+    if ((st = check_ratio(ratio)) != LOGO_OK) return st;
+    if (window < 1) return fail(LOGO_ERR_INVALID_ARG, "window=%d must be >= 1", window);
+    if ((st = resolve_scale(scale, g.d, sl2)) != LOGO_OK) return st;
+    const HostArena a = host_arena(g, ratio);
+    if (!dev_buf || !aligned16(dev_buf)) return fail(LOGO_ERR_WORKSPACE, "dev_buf is NULL or not 16-byte aligned");
+    if (dev_buf_bytes < a.total)
+        return fail(LOGO_ERR_WORKSPACE, "dev_buf of %zu bytes, the host-buffer forward needs %zu", dev_buf_bytes, a.total);
+    if (g.L > 0 && (!q || !k || !v || !out || !gate))
+        return fail(LOGO_ERR_INVALID_ARG, "q, k, v, gate and out must be non-NULL host buffers");
+    const int max_sel = (int)logo::budget_count(ratio, g.max_len);
+    uint8_t* base = static_cast<uint8_t*>(dev_buf);
+    void* ws = base + a.ws;
+    float* gate_d = reinterpret_cast<float*>(base + a.gate);
+    int32_t* cu_d = g.cu ? reinterpret_cast<int32_t*>(base + a.cu) : nullptr;
+    int32_t* sel_d = reinterpret_cast<int32_t*>(base + a.sel);
+    int32_t* cu_sel_d = reinterpret_cast<int32_t*>(base + a.cu_sel);
+    cudaStream_t s0 = static_cast<cudaStream_t>(stream);
+
+    std::lock_guard<std::mutex> lock(g_host_mu);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    HostPipe* hp = nullptr;
+    if (e == cudaSuccess) e = host_pipe(dev, hp);
+    if (e != cudaSuccess) return cuda_fail(e, "host pipeline setup");
+#define LOGO_CK(call, what)                                   \
+    do {                                                      \
+        cudaError_t ce_ = (call);                             \
+        if (ce_ != cudaSuccess) return cuda_fail(ce_, what);  \
+    } while (0)
+    // Everything the caller queued on `stream` comes first.
+    LOGO_CK(cudaEventRecord(hp->start, s0), "event");
+    LOGO_CK(cudaStreamWaitEvent(hp->in, hp->start, 0), "stream wait");
+    LOGO_CK(cudaStreamWaitEvent(hp->out, hp->start, 0), "stream wait");
+    // Gate (and packed lengths) in, selection on the compute stream.
+    if (g.L > 0) LOGO_CK(cudaMemcpyAsync(gate_d, gate, (size_t)g.B * g.L * sizeof(float), cudaMemcpyHostToDevice, hp->in), "gate copy");
+    if (g.cu) LOGO_CK(cudaMemcpyAsync(cu_d, g.cu, (size_t)(g.nseq + 1) * 4, cudaMemcpyHostToDevice, hp->in), "cu_seqlens copy");
+    LOGO_CK(cudaEventRecord(hp->inputs, hp->in), "event");
+    LOGO_CK(cudaStreamWaitEvent(s0, hp->inputs, 0), "stream wait");
+    logo_shape dsh = *shape;
+    dsh.cu_seqlens = cu_d;
+    if ((st = logo_select(gate_d, &dsh, ratio, sel_d, cu_sel_d, ws, a.ws_bytes, stream)) != LOGO_OK) return st;
+    if (sel_idx || cu_sel) {
+        LOGO_CK(cudaEventRecord(hp->sel_done, s0), "event");
+        LOGO_CK(cudaStreamWaitEvent(hp->out, hp->sel_done, 0), "stream wait");
+        if (cu_sel) LOGO_CK(cudaMemcpyAsync(cu_sel, cu_sel_d, (size_t)(g.nseq + 1) * 4, cudaMemcpyDeviceToHost, hp->out), "cu_sel copy");
+        if (sel_idx && a.sel_cap > 0)
+            LOGO_CK(cudaMemcpyAsync(sel_idx, sel_d, (size_t)a.sel_cap * 4, cudaMemcpyDeviceToHost, hp->out), "sel_idx copy");
+    }
+    // One kv-head group at a time: its Q, K, V in, both branches, its O out, with
+    // the copies of neighbouring groups overlapping the kernels.
+    Geo gu = g;
+    gu.Hq = g.G;
+    gu.Hkv = 1;
+    gu.cu = cu_d;  // the kernels read the device copy of the packed offsets
+    const size_t elt = 2;
+    const size_t rowq = (size_t)g.L * g.d * elt;  // one head of one sequence
+    const int slots = g.Hkv < kHostSlots ? g.Hkv : kHostSlots;
+    for (int hk = 0; hk < g.Hkv && g.L > 0; ++hk) {
+        const int sl = hk % slots;
+        uint8_t* slot = base + a.slot0 + (size_t)sl * a.slot_bytes;
+        uint8_t* qs = slot;
+        uint8_t* os = slot + up256(a.q_bytes);
+        uint8_t* ks = os + up256(a.q_bytes);
+        uint8_t* vs = ks + up256(a.kv_bytes);
+        if (hk >= slots) LOGO_CK(cudaStreamWaitEvent(hp->in, hp->d2h[sl], 0), "stream wait");
+        LOGO_CK(copy_rows(qs, g.G * rowq, reinterpret_cast<const uint8_t*>(q) + (size_t)hk * g.G * rowq, g.Hq * rowq,
+                          g.G * rowq, g.B, cudaMemcpyHostToDevice, hp->in), "q copy");
+        LOGO_CK(copy_rows(ks, rowq, reinterpret_cast<const uint8_t*>(k) + (size_t)hk * rowq, g.Hkv * rowq, rowq, g.B,
+                          cudaMemcpyHostToDevice, hp->in), "k copy");
+        LOGO_CK(copy_rows(vs, rowq, reinterpret_cast<const uint8_t*>(v) + (size_t)hk * rowq, g.Hkv * rowq, rowq, g.B,
+                          cudaMemcpyHostToDevice, hp->in), "v copy");
+        LOGO_CK(cudaEventRecord(hp->h2d, hp->in), "event");
+        LOGO_CK(cudaStreamWaitEvent(s0, hp->h2d, 0), "stream wait");
+        if ((st = launch_local(gu, qs, ks, vs, window, sl2, os, ws, s0)) != LOGO_OK) return st;
+        if ((st = launch_global(gu, qs, ks, vs, gate_d, sel_d, cu_sel_d, max_sel, sl2, 1, os, ws, s0)) != LOGO_OK)
+            return st;
+        LOGO_CK(cudaEventRecord(hp->comp, s0), "event");
+        LOGO_CK(cudaStreamWaitEvent(hp->out, hp->comp, 0), "stream wait");
+        LOGO_CK(copy_rows(reinterpret_cast<uint8_t*>(out) + (size_t)hk * g.G * rowq, g.Hq * rowq, os, g.G * rowq,
+                          g.G * rowq, g.B, cudaMemcpyDeviceToHost, hp->out), "out copy");
+        LOGO_CK(cudaEventRecord(hp->d2h[sl], hp->out), "event");
+    }
+    // The caller's stream completes after the last copy out.
+    LOGO_CK(cudaEventRecord(hp->done, hp->out), "event");
+    LOGO_CK(cudaStreamWaitEvent(s0, hp->done, 0), "stream wait");
+#undef LOGO_CK
+    return LOGO_OK;
 }
 
 const char* logo_status_string(logo_status s)
