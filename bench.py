@@ -79,6 +79,40 @@ def decode_source_hash():
     return h.hexdigest()[:16]
 
 
+def dense_causal_comparison(logo, q, k, v, w, ws, stream, dev, peak_burst, ms_step, reps=3):
+    """The library's own dense causal attention on the same tensors: the local kernel with the
+    window at least every sequence's length, so each query attends to its whole prefix.  Run
+    after every other figure is taken; a failure is reported in the line, not raised."""
+    try:
+        import torch
+        ml = max(w.seqlens)
+        cu = None if w.cu_seqlens is None else w.cu_seqlens.to(dev)
+        tmp = torch.empty_like(q)
+
+        def run():
+            logo.local_attn(q, k, v, ml, ws, cu_seqlens=cu, max_seqlen=ml if cu is not None else None, out=tmp,
+                            stream=stream)
+
+        run()
+        logo.check(ws, stream)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record(stream)
+        for _ in range(reps):
+            run()
+        ev[1].record(stream)
+        torch.cuda.synchronize(dev)
+        logo.check(ws, stream)
+        ms = ev[0].elapsed_time(ev[1]) / reps
+        pairs = sum(n * (n + 1) // 2 for n in w.seqlens)  # per head
+        flop = 4.0 * q.shape[3] * q.shape[1] * pairs
+        tf = flop / (ms * 1e-3) / 1e12
+        return {"kernel": "attn_fwd_kernel<d, 0> with W >= every length (dense causal)", "ms": ms,
+                "tflops": tf, "frac_of_bf16_peak": tf / peak_burst, "flop": flop,
+                "logo_step_over_dense": ms_step / ms}
+    except Exception as e:  # reported, never fatal for the bench line
+        return {"error": str(e)[:300]}
+
+
 def traffic_record():
     """DRAM bytes per launch from the committed ncu summary, if taken on the current kernel source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -523,6 +557,7 @@ def main():
 
     line = None
     if rank == 0:
+        dense = dense_causal_comparison(logo, q, k, v, w, ws, stream, dev, peak_burst, ms_step)
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             cpu = cpu_baseline(w)
@@ -559,6 +594,7 @@ def main():
             "clocks": clocks,
             "wall_s_timed": t_wall,
             "cpu_baseline": cpu,
+            "comparisons": {"dense_causal": dense},
         }
         print(json.dumps(line), flush=True)
     if world > 1:
