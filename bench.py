@@ -227,9 +227,31 @@ def cpu_baseline(w, seconds_target=15.0, seed=0):
         elapsed += time.perf_counter() - t0
         done += n_tok
         n_tok = min(64, n_tok * 2)
-    return {"value": done / elapsed, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+    cores = oracle.num_threads()
+    # the same kind of sample on one thread (a few seconds)
+    single = None
+    if cores > 1:
+        oracle.set_num_threads(1)
+        try:
+            e1, d1, n1 = 0.0, 0, 1
+            while e1 < 3.0:
+                toks = [rng.randrange(w.L) for _ in range(n1)]
+                seq = [0] * (n1 * w.Hq)
+                head = [h for _ in toks for h in range(w.Hq)]
+                pos = [t for t in toks for _ in range(w.Hq)]
+                flag = [int(t in sel) for t in toks for _ in range(w.Hq)]
+                t0 = time.perf_counter()
+                oracle.rows(w.q, w.k, w.v, w.g, w.W, seq, head, pos, flag)
+                e1 += time.perf_counter() - t0
+                d1 += n1
+                n1 = min(8, n1 * 2)
+            single = {"value": d1 / e1, "unit": "tokens/s", "sample": f"{d1} tokens, {e1:.1f} s"}
+        finally:
+            oracle.set_num_threads(cores)
+    return {"value": done / elapsed, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"{done} random query tokens of the {w.name} workload (all {w.Hq} heads, local + global "
-                      f"where selected, merge), {elapsed:.1f} s of fp64 CPU work"}
+                      f"where selected, merge), {elapsed:.1f} s of fp64 CPU work",
+            "single_thread": single}
 
 
 def run_reference(args, rank, world):

@@ -70,6 +70,8 @@ def _load():
         lib.oracle_backward_rows.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = _int
+        lib.oracle_set_num_threads.argtypes = [_int]
+        lib.oracle_set_num_threads.restype = None
         _lib = lib
         return lib
 
@@ -90,6 +92,11 @@ def num_selected(ratio: float, length: int) -> int:
 
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Thread count of the following oracle calls (n >= 1)."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def select(g: torch.Tensor, ratio: float) -> torch.Tensor:

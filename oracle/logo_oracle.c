@@ -477,6 +477,17 @@ int oracle_num_threads(void)
 #endif
 }
 
+/* Sets the number of threads of the following calls (the benchmark's
+ * single-thread baseline figure); n < 1 is ignored. */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /* ---- backward pass ---------------------------------------------------- */
 
 /*
