@@ -1,7 +1,6 @@
 """Host-side logic of bench.py that the GPU run depends on, checked on the CPU with the
 library calls and CUDA events replaced by stand-ins: the dense-causal comparison's FLOP
 count and its never-fatal error path, and the CPU baseline's single-thread figure."""
-import sys
 import types
 
 import pytest
