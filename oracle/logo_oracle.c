@@ -600,17 +600,22 @@ int64_t oracle_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         total += ks;
         /* per row and head: <dout, global>, for the gate gradient */
         double *gdot = (double *)calloc((size_t)(len * Hq), sizeof(double));
-        /* key/value heads are independent; the query heads of a group share dk, dv */
+        /* Key/value heads one after another.  Within a head, the (query head, row)
+         * pairs of its group are independent except for the sums into dk and dv,
+         * which each thread accumulates in a private copy; the copies are added
+         * into dk, dv at the end (the same sums, in another fp64 order). */
+        for (int hk = 0; hk < Hkv; ++hk) {
+            const uint16_t *kh = row_ptr(k, b, Hkv, hk, L, s0, d);
+            const uint16_t *vh = row_ptr(v, b, Hkv, hk, L, s0, d);
+            double *dkh = dk + ((b * Hkv + hk) * L + s0) * (int64_t)d;
+            double *dvh = dv + ((b * Hkv + hk) * L + s0) * (int64_t)d;
 #pragma omp parallel
-        {
-            double *p = (double *)malloc(sizeof(double) * (size_t)len);
-            double *o = (double *)malloc(sizeof(double) * (size_t)d);
-#pragma omp for schedule(dynamic, 1)
-            for (int hk = 0; hk < Hkv; ++hk) {
-                const uint16_t *kh = row_ptr(k, b, Hkv, hk, L, s0, d);
-                const uint16_t *vh = row_ptr(v, b, Hkv, hk, L, s0, d);
-                double *dkh = dk + ((b * Hkv + hk) * L + s0) * (int64_t)d;
-                double *dvh = dv + ((b * Hkv + hk) * L + s0) * (int64_t)d;
+            {
+                double *p = (double *)malloc(sizeof(double) * (size_t)len);
+                double *o = (double *)malloc(sizeof(double) * (size_t)d);
+                double *dkp = (double *)calloc((size_t)(len * d), sizeof(double));
+                double *dvp = (double *)calloc((size_t)(len * d), sizeof(double));
+#pragma omp for schedule(dynamic, 16) collapse(2)
                 for (int h = hk * G; h < (hk + 1) * G; ++h) {
                     for (int64_t i = 0; i < len; ++i) {
                         const uint16_t *qr = row_ptr(q, b, Hq, h, L, s0 + i, d);
@@ -619,20 +624,29 @@ int64_t oracle_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                         int64_t j_lo = i - W + 1;
                         if (j_lo < 0) j_lo = 0;
                         row_probs(qr, kh, vh, j_lo, i, d, pr.scale, p, o);
-                        row_grad(qr, kh, vh, er, 1.0, j_lo, i, d, pr.scale, p, o, dqr, dkh, dvh, -1);
+                        row_grad(qr, kh, vh, er, 1.0, j_lo, i, d, pr.scale, p, o, dqr, dkp, dvp, -1);
                         if (flag[i]) {
                             double a = sigmoid((double)g[b * L + s0 + i]);
                             row_probs(qr, kh, vh, 0, i, d, pr.scale, p, o);
-                            row_grad(qr, kh, vh, er, a, 0, i, d, pr.scale, p, o, dqr, dkh, dvh, -1);
+                            row_grad(qr, kh, vh, er, a, 0, i, d, pr.scale, p, o, dqr, dkp, dvp, -1);
                             double e = 0.0;
                             for (int c = 0; c < d; ++c) e += bf16_bits_to_double(er[c]) * o[c];
                             gdot[i * Hq + h] = e;
                         }
                     }
                 }
+#pragma omp critical
+                {
+                    for (int64_t x = 0; x < len * d; ++x) {
+                        dkh[x] += dkp[x];
+                        dvh[x] += dvp[x];
+                    }
+                }
+                free(dvp);
+                free(dkp);
+                free(p);
+                free(o);
             }
-            free(p);
-            free(o);
         }
         for (int64_t i = 0; i < len; ++i) {
             if (!flag[i]) continue;

@@ -51,8 +51,8 @@ MUTANTS = {
     "bwd_drop_D": ("double ds = pj * (dp - D);", "double ds = pj * dp;"),
     "bwd_gate_no_derivative": ("dg[b * L + s0 + i] = sg * (1.0 - sg) * e;", "dg[b * L + s0 + i] = sg * e;"),
     "bwd_global_upstream_ungated": (
-        "row_grad(qr, kh, vh, er, a, 0, i, d, pr.scale, p, o, dqr, dkh, dvh, -1);",
-        "row_grad(qr, kh, vh, er, 1.0, 0, i, d, pr.scale, p, o, dqr, dkh, dvh, -1);"),
+        "row_grad(qr, kh, vh, er, a, 0, i, d, pr.scale, p, o, dqr, dkp, dvp, -1);",
+        "row_grad(qr, kh, vh, er, 1.0, 0, i, d, pr.scale, p, o, dqr, dkp, dvp, -1);"),
     "bwd_dk_unscaled": ("if (dkr) dkr[c] += scale * ds * bf16_bits_to_double(q[c]);",
                         "if (dkr) dkr[c] += ds * bf16_bits_to_double(q[c]);"),
     "bwd_dv_drops_gate_factor": ("if (dvr) dvr[c] += pj * a * bf16_bits_to_double(dout[c]);",
@@ -60,11 +60,15 @@ MUTANTS = {
     "bwd_dq_reads_v": ("dq[c] += scale * ds * bf16_bits_to_double(kr[c]);",
                        "dq[c] += scale * ds * bf16_bits_to_double(vr[c]);"),
     "bwd_local_drops_self_key": (
-        "row_grad(qr, kh, vh, er, 1.0, j_lo, i, d, pr.scale, p, o, dqr, dkh, dvh, -1);",
-        "row_grad(qr, kh, vh, er, 1.0, j_lo, i > j_lo ? i - 1 : i, d, pr.scale, p, o, dqr, dkh, dvh, -1);"),
+        "row_grad(qr, kh, vh, er, 1.0, j_lo, i, d, pr.scale, p, o, dqr, dkp, dvp, -1);",
+        "row_grad(qr, kh, vh, er, 1.0, j_lo, i > j_lo ? i - 1 : i, d, pr.scale, p, o, dqr, dkp, dvp, -1);"),
     "bwd_gqa_first_head_only": (
-        "for (int h = hk * G; h < (hk + 1) * G; ++h) {\n                    for (int64_t i = 0; i < len; ++i) {",
-        "for (int h = hk * G; h < hk * G + 1; ++h) {\n                    for (int64_t i = 0; i < len; ++i) {"),
+        "for (int h = hk * G; h < (hk + 1) * G; ++h) {\n                    for (int64_t i = 0; i < len; ++i) {\n"
+        "                        const uint16_t *qr = row_ptr(q, b, Hq, h, L, s0 + i, d);\n"
+        "                        const uint16_t *er",
+        "for (int h = hk * G; h < hk * G + 1; ++h) {\n                    for (int64_t i = 0; i < len; ++i) {\n"
+        "                        const uint16_t *qr = row_ptr(q, b, Hq, h, L, s0 + i, d);\n"
+        "                        const uint16_t *er"),
 }
 
 PINS = [
