@@ -201,8 +201,14 @@ LOGO_API logo_status logo_local_attn(const logo_bf16 *q, const logo_bf16 *k, con
  * bound on every sequence's count cu_sel[s+1] - cu_sel[s] (for lists written
  * by logo_select: logo_num_selected(ratio, longest sequence)); it sizes the
  * launch, and counts above it are an error the kernel reports in the status
- * word.  sel_idx entries must be ascending within a sequence and in
- * [0, L_s).
+ * word.  sel_idx entries must be strictly ascending within a sequence and in
+ * [0, L_s).  The kernel checks what it reads: a 128-row chunk of a list whose
+ * first or last entry lies outside [0, L_s) is skipped whole, and an entry
+ * that is not above the one before it (or outside its chunk's range) is
+ * skipped alone; either sets LOGO_ERR_INVALID_ARG in the status word
+ * (logo_check) and writes nothing for the skipped rows.  A negative
+ * cu_sel[s] or a decreasing cu_sel is reported the same way.  What the kernel
+ * cannot see is the capacity of sel_idx: cu_sel must not point past it.
  */
 LOGO_API logo_status logo_global_attn_sparse(const logo_bf16 *q, const logo_bf16 *k, const logo_bf16 *v,
                                     const float *gate, const int32_t *sel_idx, const int32_t *cu_sel,
@@ -262,8 +268,10 @@ LOGO_API logo_status logo_forward_host(const logo_bf16 *q, const logo_bf16 *k, c
  * the library, held on every GPU that loads the library until exit.  Shapes
  * whose workspace (logo_workspace_size at ratio 1) exceeds it are refused with
  * LOGO_ERR_WORKSPACE.  The first call on a device looks the array's address up
- * (once per device, with that device current): make it before any stream
- * capture.  All calls on a device share the array; each call clears its
+ * (once per device, with that device current) and remembers the context it
+ * belongs to; after a device reset (a new primary context) the next call looks
+ * it up again.  Make the first call, and the first call after a reset, before
+ * any stream capture.  All calls on a device share the array; each call clears its
  * status word first, and calls that overlap on the GPU race on it.  Device
  * errors of a call are recorded there but cannot be read back: use
  * logo_global_attn_sparse and logo_check when that report is needed.  This

@@ -155,11 +155,11 @@ __device__ Work make_work(const AttnParams& p)
     } else {
         w.sel_base = p.cu_sel[seq];
         const int k = p.cu_sel[seq + 1] - w.sel_base;
-        if (k > p.max_selected) {
+        if (k > p.max_selected || k < 0 || w.sel_base < 0) {
             if (threadIdx.x == 0) atomicOr(p.status, kStatusBadArgument);
             return w;
         }
-        if (k <= 0) return w;
+        if (k == 0) return w;
         if (p.lse && p.cu_sel[seq + 1] > p.sel_stride) {
             if (threadIdx.x == 0) atomicOr(p.status, kStatusBadArgument);
             return w;
@@ -187,6 +187,13 @@ __device__ Work make_work(const AttnParams& p)
         w.max_pos = w.min_pos;
         for (int i = 0; i < kNumQ; ++i)
             if (w.nrows[i] > 0) w.max_pos = max(w.max_pos, sel[w.row0[i] + w.nrows[i] - 1]);
+        // The list comes from the caller: a tile whose first or last position lies
+        // outside the sequence is reported and skipped whole (its key range would be
+        // meaningless).  Single rows out of order are caught where they are read.
+        if (w.min_pos < 0 || w.max_pos >= w.len) {
+            if (threadIdx.x == 0) atomicOr(p.status, kStatusBadArgument);
+            return w;
+        }
         w.kv_lo = 0;
     }
     w.hk = w.head[0] / p.G;
@@ -404,14 +411,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         // Per-tile fields picked with selects (no dynamic indexing into Work).
         const int my_nrows = wg ? w.nrows[1] : w.nrows[0];
         const int my_row0 = wg ? w.row0[1] : w.row0[0];
-        const bool row_valid = r < my_nrows;
+        bool row_valid = r < my_nrows;
         const int head = wg ? w.head[1] : w.head[0];
         const int zq = w.b * p.Hq + head;
         int pos;  // position of this row within its sequence
         if (MODE == kModeLocal) {
             pos = row_valid ? my_row0 + r : w.max_pos;
         } else {
-            pos = row_valid ? p.sel_idx[w.sel_base + my_row0 + r] : w.max_pos;
+            pos = w.max_pos;
+            if (row_valid) {
+                // Each entry must lie in [min_pos, max_pos] of its tile (so inside the
+                // sequence and inside the tile's key range) and above the entry before
+                // it; a row that breaks this is reported and neither read nor written.
+                const int idx = my_row0 + r;
+                const int32_t* sel = p.sel_idx + w.sel_base;
+                const int x = sel[idx];
+                const bool ok_row = x >= w.min_pos && x <= w.max_pos && (idx == 0 || x > sel[idx - 1]);
+                if (ok_row) {
+                    pos = x;
+                } else {
+                    row_valid = false;
+                    if (half == 0) atomicOr(p.status, kStatusBadArgument);
+                }
+            }
             // Gather this half of the row of Q into the 128B-swizzled tile.
             uint8_t* dst = sQ + wg * Geo::kQBytes;
             const int4* src = reinterpret_cast<const int4*>(p.q + ((size_t)zq * p.L + w.s0 + pos) * D);
