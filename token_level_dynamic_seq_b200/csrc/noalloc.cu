@@ -13,13 +13,15 @@
 // Every GPU that loads the library holds it until the process exits.  Host
 // code cannot use the array's name as a device address, so the first call on
 // each device (with that device current) looks the address up once with
-// cudaGetSymbolAddress and caches it; make that first call before any stream
-// capture.  Every call on a device shares the one array and finds the previous
+// cudaGetSymbolAddress and caches it with the context it belongs to (a device
+// reset makes the next call look it up again); make that first call, and the
+// first call after a reset, before any stream capture.  Every call on a device shares the one array and finds the previous
 // call's contents in it: each call clears the status word first, and two
 // calls that overlap on the GPU (different streams, no ordering) race on it.
 // Device-side errors of a call land in that shared status word, which this
 // entry point does not read back: callers that need the report use
 // logo_global_attn_sparse with their own workspace and logo_check.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -37,8 +39,32 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
 
-// Device address of the static scratch on the current device (looked up once per device).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The calling thread's current context (nullptr when none is current or the
+// driver entry point is unavailable).
+CUcontext current_context()
+{
+    static std::once_flag once;
+    static CtxGetCurrentFn fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    CUcontext c = nullptr;
+    if (fn && fn(&c) != CUDA_SUCCESS) c = nullptr;
+    return c;
+}
+
+// Device address of the static scratch on the current device, looked up once
+// per device and context: after a cudaDeviceReset the runtime creates a new
+// primary context on the next call, the array lives at a new address there,
+// and the changed context handle makes this look it up again.
 logo_status scratch_address(void** out)
 {
     int dev = -1;
@@ -52,15 +78,17 @@ logo_status scratch_address(void** out)
         return LOGO_ERR_UNSUPPORTED;
     }
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_addr[dev]) {
+    const CUcontext ctx = current_context();
+    if (!g_scratch_addr[dev] || !ctx || ctx != g_scratch_ctx[dev]) {
         void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // also makes the primary context current
         if (e != cudaSuccess || !p) {
             logo::set_last_error("no-alloc scratch: cudaGetSymbolAddress failed on device %d: %s", dev,
                                  cudaGetErrorString(e));
             return LOGO_ERR_CUDA;
         }
         g_scratch_addr[dev] = p;
+        g_scratch_ctx[dev] = current_context();
     }
     *out = g_scratch_addr[dev];
     return LOGO_OK;
