@@ -285,6 +285,8 @@ def test_select_random_ties_specials(seed):
 # --------------------------------------------------------------------------
 
 def sampled_rows(w, sel_lists_, n_random=192, n_sel=96, seed=0):
+    """Random rows (any head, any position; and selected positions), plus both ends of the last
+    sequence."""
     rng = random.Random(seed)
     rows = []
     nonempty = [s for s, n in enumerate(w.seqlens) if n > 0]
@@ -301,12 +303,53 @@ def sampled_rows(w, sel_lists_, n_random=192, n_sel=96, seed=0):
     return rows
 
 
-def check_sampled(w, out, sel_lists_, seed=0):
-    rows = sampled_rows(w, sel_lists_, seed=seed)
+def cta_query_tiles(w, sel_lists_):
+    """The query tiles of every CTA of the two forward launches, in the kernels' own decomposition.
+
+    A CTA owns two 128-row query tiles that read one key/value head: with an even group size
+    two heads (2p, 2p+1) on the same rows (local: rows [t0, t0+128); global: list entries
+    [c0, c0+128) of one sequence), otherwise two consecutive 128-row tiles of one head.
+    Yields (kind, seq, head, lo, hi) with [lo, hi) a range of positions (local) or of
+    indices into the sequence's selection list (global)."""
+    G = w.Hq // w.Hkv
+    pair = G % 2 == 0
+    unit = 128 if pair else 256
+    for s, n in enumerate(w.seqlens):
+        for kind, count in (("local", n), ("global", len(sel_lists_[s]))):
+            for c0 in range(0, count, unit):
+                if pair:
+                    tiles = [(h, c0, min(count, c0 + 128)) for h in range(w.Hq)]
+                else:
+                    tiles = [(h, a, min(count, a + 128)) for h in range(w.Hq) for a in (c0, c0 + 128) if a < count]
+                for h, lo, hi in tiles:
+                    yield kind, s, h, lo, hi
+
+
+def cta_rows(w, sel_lists_, n_inner=1, seed=0, kinds=("local", "global")):
+    """Rows that reach every CTA of the forward launches named in `kinds`: for each query tile of
+    each CTA its first row, its last row and `n_inner` rows drawn inside it (local tiles:
+    positions; global tiles: entries of the selection list)."""
+    rng = random.Random(seed)
+    rows = set()
+    for kind, s, h, lo, hi in cta_query_tiles(w, sel_lists_):
+        if kind not in kinds:
+            continue
+        picks = [lo, hi - 1] + [rng.randrange(lo, hi) for _ in range(n_inner)]
+        for x in picks:
+            rows.add((s, h, x if kind == "local" else sel_lists_[s][x]))
+    return sorted(rows)
+
+
+def check_rows(w, out, sel_lists_, rows, what, local_only=False):
+    """Compare the given (seq, head, position) rows of `out` with the oracle, which computes
+    each row on its own: the local branch, the global branch where selected, the merge; or,
+    with `local_only`, the local branch alone (`out` then holds logo_local_attn's output)."""
     sets = [set(x) for x in sel_lists_]
+    flags = [0 if local_only else int(r[2] in sets[r[0]]) for r in rows]
     loc, glo, ref = oracle.rows(w.q, w.k, w.v, w.g, w.W, [r[0] for r in rows], [r[1] for r in rows],
-                                [r[2] for r in rows], [int(r[2] in sets[r[0]]) for r in rows],
-                                cu_seqlens=w.cu_seqlens)
+                                [r[2] for r in rows], flags, cu_seqlens=w.cu_seqlens)
+    if local_only:
+        ref = loc
     outc = out.cpu()
     got = []
     for s, h, i in rows:
@@ -314,7 +357,24 @@ def check_sampled(w, out, sel_lists_, seed=0):
             got.append(outc[s, h, i])
         else:
             got.append(outc[0, h, int(w.cu_seqlens[s]) + i])
-    return close(torch.stack(got), ref, f"{w.name} sampled")
+    return close(torch.stack(got), ref, f"{what} ({len(rows)} rows)")
+
+
+def check_sampled(w, out, sel_lists_, seed=0):
+    return check_rows(w, out, sel_lists_, sampled_rows(w, sel_lists_, seed=seed), f"{w.name} sampled")
+
+
+def check_every_cta(w, out, sel_lists_, n_inner=1, seed=0, local_out=None):
+    """Rows reaching every CTA of both launches.  With `local_out` (logo_local_attn's output on
+    the same inputs) the local launch's rows are compared branch by branch, which spares the
+    oracle the whole-prefix branch of the selected ones; otherwise every row is compared merged."""
+    if local_out is None:
+        return check_rows(w, out, sel_lists_, cta_rows(w, sel_lists_, n_inner=n_inner, seed=seed),
+                          f"{w.name} every CTA")
+    check_rows(w, local_out, sel_lists_, cta_rows(w, sel_lists_, n_inner, seed, kinds=("local",)),
+               f"{w.name} every local CTA (local branch)", local_only=True)
+    return check_rows(w, out, sel_lists_, cta_rows(w, sel_lists_, n_inner, seed, kinds=("global",)),
+                      f"{w.name} every global CTA (merged)")
 
 
 def run_full(w):
@@ -337,14 +397,34 @@ def test_named_small_full(name):
 
 
 @pytest.mark.parametrize("name", ["c32k", "varlen"])
-def test_named_large_sampled(name):
+def test_named_large_every_cta(name):
+    """Full size, benchmark launch configuration: the selection in full, and rows that reach
+    every CTA of the local and the global launch (first, last and one inner row of each of a
+    CTA's query tiles), plus a random sample."""
     w = workloads.load(name)
     out, lists, _ = run_full(w)
     assert lists == oracle_sel_lists(w)
+    check_every_cta(w, out, lists)
     check_sampled(w, out, lists)
 
 
-def test_c128k_ratio_sweep_sampled():
+def test_c32k_one_group_in_full():
+    """Headline size: every element of one key/value-head group's output (its 4 query heads,
+    all 32768 rows) against the oracle run on that group alone.  A group is an independent
+    problem once the selection is fixed, and the selection depends on the gate only."""
+    w = workloads.load("c32k")
+    out, lists, _ = run_full(w)
+    G = w.Hq // w.Hkv
+    hk = w.Hkv - 1
+    ref = oracle.forward(w.q[:, hk * G:(hk + 1) * G].contiguous(), w.k[:, hk:hk + 1].contiguous(),
+                         w.v[:, hk:hk + 1].contiguous(), w.g, w.W, w.ratio)
+    assert ref["sel_idx"].tolist() == lists[0]
+    close(out[:, hk * G:(hk + 1) * G], ref["out"], f"c32k group {hk} in full")
+
+
+def test_c128k_ratio_sweep():
+    """L = 131072 at every ratio of the sweep: the selection in full and a random row sample;
+    at ratio 0.2 also rows that reach every CTA of both launches."""
     base = workloads.load("c128k_r0.2")
     for r in workloads.RATIO_SWEEP_128K:
         base.ratio = r
@@ -352,6 +432,14 @@ def test_c128k_ratio_sweep_sampled():
         out, lists, _ = run_full(base)
         assert lists == oracle_sel_lists(base)
         check_sampled(base, out, lists, seed=int(r * 100))
+        if r == 0.2:
+            q, k, v, _, _ = to_dev(base)
+            ws = logo.workspace(logo.make_shape(q, k), base.ratio, q.device)
+            loc = logo.local_attn(q, k, v, base.W, ws)
+            logo.check(ws)
+            del q, k, v
+            check_every_cta(base, out, lists, n_inner=0, local_out=loc)
+            del loc
         del out
         torch.cuda.empty_cache()
 
@@ -375,3 +463,78 @@ def test_timeout_is_reported_and_context_survives():
     logo.check(ws2)
     ref = oracle.forward(w.q, w.k, w.v, w.g, w.W, w.ratio)
     close(out, ref["out"], "after timeout")
+
+
+# --------------------------------------------------------------------------
+# caller-supplied selection lists that break the contract
+# --------------------------------------------------------------------------
+
+def test_global_rejects_bad_selection_lists():
+    """Lists with an entry outside the sequence, an entry out of order, a chunk whose last entry
+    lies past the sequence, or decreasing offsets: the kernel reports LOGO_ERR_INVALID_ARG through
+    the status word, neither reads nor writes the offending rows (a whole chunk when its first or
+    last entry is out of range), writes nothing outside `out`, and computes every other row
+    exactly as with the valid list."""
+    w = small_workload(("bad lists", 1, 4, 2, 600, 128, 64, 0.25, None), seed=2)
+    q, k, v, g, cu = to_dev(w)
+    L = w.L
+    shape = logo.make_shape(q, k)
+    ws = logo.workspace(shape, w.ratio, q.device)
+    sel, cu_sel = logo.select(g, shape, w.ratio, ws)
+    logo.check(ws)
+    good = sel.clone()
+    n = int(cu_sel[1])
+    assert n == 150  # two 128-entry chunks
+    kmax = n
+    pad = 4096
+
+    def run(sel_arg, cu_arg):
+        buf = torch.full((q.numel() + 2 * pad,), 7.0, dtype=torch.bfloat16, device=q.device)
+        out = buf[pad:pad + q.numel()].view_as(q)
+        ws2 = logo.workspace(shape, w.ratio, q.device)
+        logo.global_attn_sparse(q, k, v, g, sel_arg, cu_arg, kmax, out, ws2, merge=False)
+        torch.cuda.synchronize()
+        guards_ok = bool((buf[:pad] == 7.0).all()) and bool((buf[pad + q.numel():] == 7.0).all())
+        return out.cpu(), ws2, guards_ok
+
+    ref_out, ws_ok, guards = run(good, cu_sel)
+    logo.check(ws_ok)
+    assert guards
+    lst = good.cpu().tolist()
+
+    def bad_case(edit, skipped_entries, cu_arg=None):
+        b = torch.tensor(edit(list(lst)), dtype=torch.int32, device=q.device)
+        out, ws2, guards_ok = run(b, cu_sel if cu_arg is None else cu_arg)
+        with pytest.raises(logo.LogoError) as e:
+            logo.check(ws2)
+        assert e.value.status == 1
+        assert guards_ok, "a write landed outside out"
+        skipped_pos = {lst[i] for i in skipped_entries}
+        for i, pos in enumerate(lst):
+            if pos in skipped_pos:
+                assert (out[0, :, pos] == 7.0).all(), f"row {pos} of a rejected entry was written"
+            elif cu_arg is None:
+                assert torch.equal(out[0, :, pos], ref_out[0, :, pos]), f"valid row {pos} changed"
+
+    def set_(i, val):
+        def f(x):
+            x[i] = val
+            return x
+        return f
+
+    def swap(i):
+        def f(x):
+            x[i], x[i + 1] = x[i + 1], x[i]
+            return x
+        return f
+
+    # past the end in the middle of chunk 0: that entry and the next (now not above it) are skipped
+    bad_case(set_(5, L + 7), [5, 6])
+    # negative in the middle of chunk 1
+    bad_case(set_(130, -5), [130])
+    # last entry of chunk 1 past the end: the whole chunk is skipped
+    bad_case(set_(149, L), list(range(128, 150)))
+    # two entries out of order: the second (now below the first) is skipped
+    bad_case(swap(50), [50])
+    # decreasing offsets: nothing at all is computed
+    bad_case(lambda x: x, list(range(150)), cu_arg=torch.tensor([0, -1], dtype=torch.int32, device=q.device))
