@@ -45,10 +45,18 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-batch", type=int, default=64, help="sequences of the decode workload")
+    ap.add_argument("--profile", action="store_true",
+                    help="time the kernels only (no end-to-end run, dense comparison or CPU baseline): "
+                         "the lean command a profiler capture wraps")
     ap.add_argument("--shard", default="sequences", choices=["sequences", "heads"],
                     help="sequences: each rank runs its own sequence (weak scaling); heads: the ranks split one "
                          "problem by key/value-head groups (strong scaling)")
     return ap.parse_args()
+
+
+# NVIDIA's datasheet figure for dense bf16 tensor-core throughput of one B200 (the 4.5 PFLOP/s
+# they print is with 2:4 sparsity; dense is half).  Reported beside the measured matmul peak.
+DATASHEET_DENSE_BF16_TFLOPS = 2250.0
 
 
 def peaks():
@@ -77,6 +85,23 @@ def decode_source_hash():
         with open(os.path.join(ROOT, "token_level_dynamic_seq_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def algorithmic_bytes(d, Hq, Hkv, seqlens, counts, last_sel):
+    """Bytes each forward kernel must move at least once between HBM and the SMs (bf16 tensors).
+
+    Local launch: Q, K and V read once and O written once: T * d * 2 * (2 Hq + 2 Hkv).
+    Global launch, per sequence s with k_s selected tokens, the last at position p_s: the
+    selected Q rows (k_s Hq d 2), K and V up to p_s once per key/value head (2 Hkv (p_s + 1) d 2),
+    the selected rows of O read (the local branch) and written back (2 k_s Hq d 2), and the gate
+    logits and positions of the selected tokens (2 * 4 k_s)."""
+    T = sum(seqlens)
+    local = T * d * 2 * (2 * Hq + 2 * Hkv)
+    glob = 0
+    for k_s, p_s in zip(counts, last_sel):
+        if k_s > 0:
+            glob += k_s * Hq * d * 2 + 2 * Hkv * (p_s + 1) * d * 2 + 2 * k_s * Hq * d * 2 + 8 * k_s
+    return {"local": local, "global": glob}
 
 
 def dense_causal_comparison(logo, q, k, v, w, ws, stream, dev, peak_burst, ms_step, reps=3):
@@ -434,6 +459,47 @@ def run_train(args, rank, world):
         print(json.dumps(line), flush=True)
 
 
+def run_e2e(args, logo, w, hq, hk, hv, out, ml, dev, stream, world, job_tokens, ws):
+    """The same metric end to end through logo_forward_host: page-locked host buffers, the copies
+    of Q/K/V/g in and of the output and the selection out inside the timed region."""
+    from token_level_dynamic_seq_b200 import multirank
+
+    pin = [x.contiguous().pin_memory() for x in (hq, hk, hv, w.g)]
+    cu_host = None if w.cu_seqlens is None else w.cu_seqlens.contiguous().pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    nseq_h = len(w.seqlens)
+    sel_host = torch.empty(max(1, nseq_h * logo.num_selected(w.ratio, ml)), dtype=torch.int32).pin_memory()
+    cu_sel_host = torch.empty(nseq_h + 1, dtype=torch.int32).pin_memory()
+    hbuf = logo.host_buffer(logo.make_shape(pin[0], pin[1], cu_host, ml if cu_host is not None else None),
+                            w.ratio, dev, stream)
+    h2d = sum(x.numel() * x.element_size() for x in pin) + (0 if cu_host is None else cu_host.numel() * 4)
+    d2h = (out_host.numel() * out_host.element_size() + sel_host.numel() * 4 + cu_sel_host.numel() * 4)
+
+    def e2e_step():
+        logo.forward_host(*pin, w.W, w.ratio, buf=hbuf, device=dev, cu_seqlens=cu_host,
+                          max_seqlen=ml if cu_host is not None else None, out=out_host, sel_idx=sel_host,
+                          cu_sel=cu_sel_host, stream=stream)
+
+    e2e_step()  # first call creates the copy streams
+    logo.check(hbuf, stream)
+    e2e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e2e_ev[0].record(stream)
+    n_e2e = max(1, args.e2e_steps)
+    for _ in range(n_e2e):
+        e2e_step()
+    e2e_ev[1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = multirank.max_over_ranks(e2e_ev[0].elapsed_time(e2e_ev[1]) / n_e2e, device=dev)
+    logo.check(ws, stream)
+    logo.check(hbuf, stream)
+
+    return {"value": job_tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -505,6 +571,12 @@ def main():
     fl_local = 4 * w.d * Hq_r * lp
     fl_global = 4 * w.d * Hq_r * sel_pos_sum
     tokens = w.tokens
+    cu_sel_h = cu_sel.cpu().tolist()
+    sel_h = sel[:tot_sel].cpu().tolist()
+    last_sel = [sel_h[cu_sel_h[s] + n - 1] if n > 0 else -1
+                for s, n in enumerate(cu_sel_h[i + 1] - cu_sel_h[i] for i in range(nseq))]
+    alg_bytes = algorithmic_bytes(w.d, Hq_r, k.shape[1], w.seqlens, [cu_sel_h[i + 1] - cu_sel_h[i] for i in range(nseq)],
+                                  last_sel)
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     sampler = ClockSampler(local_rank)
@@ -536,52 +608,26 @@ def main():
 
     # end to end through the public API with host buffers: logo_forward_host copies the
     # page-locked inputs in and the output and selection out, inside the timed region
-    pin = [x.contiguous().pin_memory() for x in (hq, hk, hv, w.g)]
-    cu_host = None if w.cu_seqlens is None else w.cu_seqlens.contiguous().pin_memory()
-    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    nseq_h = len(w.seqlens)
-    sel_host = torch.empty(max(1, nseq_h * logo.num_selected(w.ratio, ml)), dtype=torch.int32).pin_memory()
-    cu_sel_host = torch.empty(nseq_h + 1, dtype=torch.int32).pin_memory()
-    hbuf = logo.host_buffer(logo.make_shape(pin[0], pin[1], cu_host, ml if cu_host is not None else None),
-                            w.ratio, dev, stream)
-    h2d = sum(x.numel() * x.element_size() for x in pin) + (0 if cu_host is None else cu_host.numel() * 4)
-    d2h = (out_host.numel() * out_host.element_size() + sel_host.numel() * 4 + cu_sel_host.numel() * 4)
-
-    def e2e_step():
-        logo.forward_host(*pin, w.W, w.ratio, buf=hbuf, device=dev, cu_seqlens=cu_host,
-                          max_seqlen=ml if cu_host is not None else None, out=out_host, sel_idx=sel_host,
-                          cu_sel=cu_sel_host, stream=stream)
-
-    e2e_step()  # first call creates the copy streams
-    logo.check(hbuf, stream)
-    e2e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    e2e_ev[0].record(stream)
-    n_e2e = max(1, args.e2e_steps)
-    for _ in range(n_e2e):
-        e2e_step()
-    e2e_ev[1].record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = multirank.max_over_ranks(e2e_ev[0].elapsed_time(e2e_ev[1]) / n_e2e, device=dev)
-    logo.check(ws, stream)
-    logo.check(hbuf, stream)
+    e2e = run_e2e(args, logo, w, hq, hk, hv, out, ml, dev, stream, world, job_tokens, ws) if not args.profile else None
 
     peak_burst, peak_sust, hbm, peak_src = peaks()
     dominant = "local" if avg["local"] >= avg["global"] else "global"
     dom_flops = fl_local if dominant == "local" else fl_global
     achieved = dom_flops / (avg[dominant] * 1e-3) / 1e12
-    tr = traffic_record()
-    kern_name = {"local": "attn_fwd_kernel<128, 0>", "global": "attn_fwd_kernel<128, 1>"}[dominant]
-    traffic = tr.get(kern_name, {}).get("bytes_per_launch") if isinstance(tr.get(kern_name), dict) else None
+    tr = traffic_record() if (w.name == WORKLOAD and world == 1 and not by_heads) else {}
+    names = {"local": "attn_fwd_kernel<128, 0>", "global": "attn_fwd_kernel<128, 1>"}
+    kern_name = names[dominant]
+    traffic_of = {kk: (tr.get(nm, {}).get("bytes_per_launch") if isinstance(tr.get(nm), dict) else None)
+                  for kk, nm in names.items()}
+    traffic = traffic_of[dominant]
     useful_tflops = multirank.sum_over_ranks(fl_local + fl_global, device=dev) / (ms_step * 1e-3) / 1e12
 
     line = None
     if rank == 0:
-        dense = dense_causal_comparison(logo, q, k, v, w, ws, stream, dev, peak_burst, ms_step)
+        dense = None if args.profile else dense_causal_comparison(logo, q, k, v, w, ws, stream, dev, peak_burst,
+                                                                   ms_step)
         cpu = None
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not (args.no_cpu_baseline or args.profile):
             cpu = cpu_baseline(w)
         line = {
             "metric": METRIC,
@@ -603,15 +649,22 @@ def main():
                            (q.numel() + k.numel() + v.numel() + out.numel()) * 2 / 1e6)},
             "useful_tflops": useful_tflops,
             "useful_frac_of_bf16_peak": useful_tflops / (peak_burst * world),
+            "useful_frac_of_datasheet_dense_bf16": useful_tflops / (DATASHEET_DENSE_BF16_TFLOPS * world),
             "kernels_ms": avg,
             "kernels_tflops": {"local": fl_local / (avg["local"] * 1e-3) / 1e12,
                                "global": fl_global / (avg["global"] * 1e-3) / 1e12},
             "useful_flop": {"local": fl_local, "global": fl_global},
             "roofline": {"kernel": kern_name, "bound": "tensor", "achieved": achieved, "peak": peak_burst,
                          "unit": "TFLOP/s", "frac": achieved / peak_burst, "traffic": traffic,
-                         "peak_source": f"{peak_src} bf16 burst (sustained {peak_sust})"},
-            "e2e": {"value": job_tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                         "peak_source": f"{peak_src} bf16 burst (sustained {peak_sust})",
+                         "frac_of_datasheet_dense_bf16": achieved / DATASHEET_DENSE_BF16_TFLOPS,
+                         "datasheet_source": "NVIDIA B200 dense bf16 tensor-core figure, 2.25 PFLOP/s",
+                         "algorithmic_bytes": alg_bytes[dominant],
+                         "traffic_over_algorithmic": (traffic / alg_bytes[dominant]) if traffic else None},
+            "kernels_bytes": {kk: {"algorithmic": alg_bytes[kk], "dram_traffic": traffic_of[kk],
+                                   "achieved_gbs": alg_bytes[kk] / (avg[kk] * 1e-3) / 1e9}
+                              for kk in ("local", "global")},
+            "e2e": e2e,
             "gpu_launches": 3 * args.steps,
             "clocks": clocks,
             "wall_s_timed": t_wall,
