@@ -3,10 +3,12 @@
 // except in logo_check.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -18,6 +20,32 @@ namespace {
 using logo::AttnParams;
 
 thread_local char g_last_error[512] = "";
+
+// NVTX ranges around each kernel launch, for a profiler's timeline.  Off unless
+// the environment sets LOGO_NVTX=1 when the library first launches something;
+// NVTX itself does nothing unless a tool has injected its library.
+bool nvtx_on()
+{
+    static const bool on = [] {
+        const char* e = std::getenv("LOGO_NVTX");
+        return e && e[0] == '1';
+    }();
+    return on;
+}
+
+struct NvtxRange {
+    const bool on;
+    explicit NvtxRange(const char* name) : on(nvtx_on())
+    {
+        if (on) nvtxRangePushA(name);
+    }
+    ~NvtxRange()
+    {
+        if (on) nvtxRangePop();
+    }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 logo_status fail(logo_status s, const char* fmt, ...)
 {
@@ -191,6 +219,7 @@ logo_status launch_local(const Geo& g, const void* q, const void* k, const void*
     if ((st = make_map(&p.tm_q, q, g.d, g.L, g.B * g.Hq)) != LOGO_OK) return st;
     if ((st = make_map(&p.tm_k, k, g.d, g.L, g.B * g.Hkv)) != LOGO_OK) return st;
     if ((st = make_map(&p.tm_v, v, g.d, g.L, g.B * g.Hkv)) != LOGO_OK) return st;
+    NvtxRange range("logo local attention");
     cudaError_t e = logo::launch_attn(logo::kModeLocal, g.d, p, g.max_len, stream);
     if (e != cudaSuccess) return cuda_fail(e, "local attention launch");
     return LOGO_OK;
@@ -218,6 +247,7 @@ logo_status launch_global(const Geo& g, const void* q, const void* k, const void
     logo_status st;
     if ((st = make_map(&p.tm_k, k, g.d, g.L, g.B * g.Hkv)) != LOGO_OK) return st;
     if ((st = make_map(&p.tm_v, v, g.d, g.L, g.B * g.Hkv)) != LOGO_OK) return st;
+    NvtxRange range("logo selected-query global attention");
     cudaError_t e = logo::launch_attn(logo::kModeGlobal, g.d, p, g.max_len, stream);
     if (e != cudaSuccess) return cuda_fail(e, "global attention launch");
     return LOGO_OK;
@@ -374,6 +404,7 @@ logo_status logo_select(const float* gate, const logo_shape* shape, double ratio
     if (g.L == 0 && !g.cu) {
         e = cudaMemsetAsync(cu_sel, 0, sizeof(int32_t) * (size_t)(g.nseq + 1), static_cast<cudaStream_t>(stream));
     } else {
+        NvtxRange range("logo select");
         e = logo::launch_select(gate, g.cu, g.nseq, g.L, ratio, sel_idx, cu_sel, static_cast<cudaStream_t>(stream));
     }
     return e == cudaSuccess ? LOGO_OK : cuda_fail(e, "select launch");
@@ -561,6 +592,7 @@ logo_status logo_backward(const logo_bf16* q, const logo_bf16* k, const logo_bf1
     pp.L = g.L;
     pp.nseq = g.nseq;
     pp.sel_stride = any_sel ? sel_capacity : 0;
+    NvtxRange range("logo backward");
     cudaError_t e = logo::launch_bwd_prep(pp, g.d, s);
     if (e != cudaSuccess) return cuda_fail(e, "backward prep launch");
 
@@ -625,6 +657,7 @@ logo_status logo_select_threshold(const float* gate, const logo_shape* shape, co
     if (max_selected > 0 && (st = check_ptr(sel_idx, "sel_idx")) != LOGO_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int32_t* counts = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kWsHeaderBytes);
+    NvtxRange range("logo threshold select");
     cudaError_t e = logo::launch_threshold_select(gate, g.cu, g.nseq, g.L, tau, max_selected, counts, sel_idx, cu_sel,
                                                   static_cast<uint32_t*>(ws), s);
     return e == cudaSuccess ? LOGO_OK : cuda_fail(e, "threshold select launch");
@@ -644,6 +677,7 @@ logo_status logo_threshold_update(const float* gate, const logo_shape* shape, do
         return fail(LOGO_ERR_INVALID_ARG, "target is not 4-byte aligned");
     if (g.L > 0 && (st = check_ptr(gate, "gate")) != LOGO_OK) return st;
     const long long n_fixed = (long long)g.B * g.L;
+    NvtxRange range("logo threshold update");
     cudaError_t e = logo::launch_threshold_update(gate, g.cu, g.nseq, n_fixed, ratio, beta, tau, target,
                                                   static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? LOGO_OK : cuda_fail(e, "threshold update launch");
@@ -709,6 +743,7 @@ logo_status logo_decode(const logo_bf16* q, const logo_bf16* k_cache, const logo
             (st = make_map_box(&p.tm_v, v_cache, g.d, g.L, g.B * g.Hkv, logo::kDecBlock)) != LOGO_OK)
             return st;
     }
+    NvtxRange range("logo decode");
     cudaError_t e = logo::launch_decode(p, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? LOGO_OK : cuda_fail(e, "decode launch");
 }

@@ -17,14 +17,17 @@
 // consecutive row tiles of one head.  Each key/value tile is staged once in
 // shared memory by TMA and feeds both query tiles.
 //
-// Warp roles (18 warps):
+// Warp roles (12 warps, three warpgroups):
 //   warp 0       TMA producer: Q tiles (local mode) and the K/V ring.
 //   warp 1       tcgen05 issuer (one thread): S_i = Q_i K^T into TMEM, then
 //                O_i += P_i V with P_i read straight from TMEM.
-//   warps 2-9    softmax for query tile 0: two warpgroups, one per half of the
-//                128 key columns (thread = row = TMEM lane); the halves meet
-//                once per tile to combine their row maxima
-//   warps 10-17  the same for query tile 1
+//   warps 2-3    idle; with warps 0-1 they form the producer warpgroup, which
+//                hands most of its registers to the softmax warpgroups
+//                (setmaxnreg: 56 registers per thread there, 224 in the softmax).
+//   warps 4-7    softmax for query tile 0: thread = row = TMEM lane, holding all
+//                128 scores of its row, so the row maximum is a thread-local
+//                reduction.
+//   warps 8-11   the same for query tile 1.
 // TMEM (512 columns): S_0 | S_1 | O_0 | O_1.  P_i (bf16 pairs) overwrites the
 // first half of S_i once the row has been read into registers.
 //
@@ -37,9 +40,9 @@
 //   after PV_i(j) has read them, because tcgen05 MMAs from one thread execute
 //   in issue order; and the commit that signals S_i(j+1) also covers
 //   PV_i(j), so O_i may be rescaled as soon as S_i(j+1) is seen.  P_i(j) is
-//   published in two parts (one per half-row warpgroup) and the MMAs of the
-//   first part write all of O_i, so only the first half's warpgroup rescales
-//   O_i (every column), before it publishes its part.
+//   published in two parts (keys 0-63, then 64-127) and the MMAs of the first
+//   part write all of O_i, so a rescale of O_i happens before the first part
+//   is published.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -51,28 +54,15 @@
 
 namespace logo {
 
+
 namespace {
 
 constexpr int kKStages = 2;
 constexpr int kVStages = 2;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
-#ifndef LOGO_P_PARTS
-#define LOGO_P_PARTS 2
-#endif
-// P_i is published in kPParts column blocks; the PV MMAs of a block start
-// while the softmax computes the next one.
-constexpr int kPParts = LOGO_P_PARTS;
-static_assert(kPParts == 2, "P is published in two parts, one per half-row warpgroup");
-#ifndef LOGO_POLY_EVERY
-#define LOGO_POLY_EVERY 0
-#endif
-// Every kPolyEvery-th pair of exponentials of a row uses exp2_poly2 (FMA pipe)
-// instead of the MUFU unit; 0 keeps them all on MUFU.
-constexpr int kPolyEvery = LOGO_POLY_EVERY;
-__device__ __forceinline__ constexpr bool use_poly(int pair)
-{
-    return kPolyEvery > 0 && (pair % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
-}
+// P_i is published in two column blocks (keys 0-63, then 64-127): the PV MMAs of
+// the first start while the softmax computes the second.
+constexpr int kPParts = 2;
 
 template <int D>
 struct Geometry {
@@ -84,9 +74,8 @@ struct Geometry {
     static constexpr int kKOff = kQOff + kNumQ * kQBytes;
     static constexpr int kVOff = kKOff + kKStages * kKVBytes;
     static constexpr int kBarOff = kVOff + kVStages * kKVBytes;
-    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + (2 + kPParts) * kNumQ + 2;
-    static constexpr int kXchgOff = kBarOff + kNumBars * 8 + 16;      // [kNumQ][2][128] floats
-    static constexpr int kBytes = kXchgOff + kNumQ * 2 * 128 * 4;
+    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + (1 + kPParts) * kNumQ + 2;
+    static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
     static constexpr int kTmemS = 0;          // S_i at column 128 * i
     static constexpr int kTmemO = 128 * kNumQ; // O_i at column 256 + D * i
     static constexpr uint32_t kTmemCols = 512;
@@ -225,11 +214,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     uint64_t* s_full = v_empty + kVStages;
     uint64_t* p_full = s_full + kNumQ;        // [kNumQ][kPParts]: part k of P_i written
     uint64_t* o_full = p_full + kPParts * kNumQ;
-    uint64_t* pair_bar = o_full + 1;          // [kNumQ]: the two halves of a row meet (256 arrivals)
-    uint64_t* drain = pair_bar + kNumQ;
+    uint64_t* drain = o_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    float* xchg = reinterpret_cast<float*>(smem + Geo::kXchgOff);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -245,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     if (!w.valid) return;  // uniform across the CTA
 
     if (threadIdx.x == 0) {
-        mbar_init(q_full, MODE == kModeLocal ? 1 : 256 * kNumQ);
+        mbar_init(q_full, MODE == kModeLocal ? 1 : 128 * kNumQ);
         for (int s = 0; s < kKStages; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
@@ -257,7 +244,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         for (int i = 0; i < kNumQ; ++i) mbar_init(&s_full[i], 1);
         for (int i = 0; i < kPParts * kNumQ; ++i) mbar_init(&p_full[i], 128);
         mbar_init(o_full, 1);
-        for (int i = 0; i < kNumQ; ++i) mbar_init(&pair_bar[i], 256);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -274,7 +260,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const int n_kv = w.n_kv;
     const int zkv = w.b * p.Hkv + w.hk;
 
-    if (warp == 0) {
+    if (warp < 4) {
+      // Producer warpgroup: TMA (warp 0), tcgen05 issue (warp 1), two idle warps.
+      // It hands registers to the softmax warpgroups.
+      reg_dealloc<kProducerRegs>();
+      if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch_desc(&p.tm_k);
@@ -391,23 +381,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             volatile int dummy = 0;
             mbar_wait(drain, 0, &dummy, nullptr, limit);
         }
+      }
     } else {
+        reg_alloc<kSoftmaxRegs>();
         // ------------------------------------------------------------ softmax warpgroups
-        // Four warpgroups: two per query tile, each owning 64 of the 128 columns
-        // of every row (thread = row = TMEM lane).  The two halves of a row meet
-        // once per tile to combine their maxima (and once at the end for the sums).
-        const int sw = (warp - 2) >> 2;          // softmax warpgroup 0..3
-        const int wg = sw >> 1;                   // query tile
-        const int half = sw & 1;                  // columns 64*half .. 64*half+63 of S_wg
+        // One warpgroup per query tile; thread = row = TMEM lane, holding all 128
+        // scores of its row, so the row maximum needs no exchange.
+        const int wg = (warp - 4) >> 2;           // query tile
         const int quarter = warp & 3;             // TMEM lane quarter this warp may touch
         const int r = quarter * 32 + lane;        // row of the tile = TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const uint32_t tS = tmem + lane_off + Geo::kTmemS + 128 * wg + 64 * half;  // this half's S
-        const uint32_t tP = tmem + lane_off + Geo::kTmemS + 128 * wg + 32 * half;  // this half's P
-        const uint32_t tO_row = tmem + lane_off + Geo::kTmemO + D * wg;  // all D columns of O for this row
-        const uint32_t tO = tO_row + (D / 2) * half;                       // this half's D/2 columns
-        float* xch = xchg + (wg * 2) * 128;       // [2][128]: one value per row from each half
-        uint64_t* pair = &pair_bar[wg];
+        const uint32_t tS = tmem + lane_off + Geo::kTmemS + 128 * wg;  // S_wg, and P_wg over its first 64 columns
+        const uint32_t tO = tmem + lane_off + Geo::kTmemO + D * wg;    // all D columns of O for this row
         // Per-tile fields picked with selects (no dynamic indexing into Work).
         const int my_nrows = wg ? w.nrows[1] : w.nrows[0];
         const int my_row0 = wg ? w.row0[1] : w.row0[0];
@@ -431,16 +416,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     pos = x;
                 } else {
                     row_valid = false;
-                    if (half == 0) atomicOr(p.status, kStatusBadArgument);
+                    atomicOr(p.status, kStatusBadArgument);
                 }
             }
-            // Gather this half of the row of Q into the 128B-swizzled tile.
+            // Gather this row of Q into the 128B-swizzled tile.
             uint8_t* dst = sQ + wg * Geo::kQBytes;
             const int4* src = reinterpret_cast<const int4*>(p.q + ((size_t)zq * p.L + w.s0 + pos) * D);
-            constexpr int kUnits = Geo::kChunks * 8 / 2;  // 16-byte units per half row
+            constexpr int kUnits = Geo::kChunks * 8;  // 16-byte units per row
             #pragma unroll
-            for (int uu = 0; uu < kUnits; ++uu) {
-                const int u = half * kUnits + uu;
+            for (int u = 0; u < kUnits; ++u) {
                 const int c = u >> 3, e = u & 7;
                 const int4 val = row_valid ? __ldg(src + u) : make_int4(0, 0, 0, 0);
                 *reinterpret_cast<int4*>(dst + c * Geo::kChunkBytes + r * 128 + ((e ^ (r & 7)) << 4)) = val;
@@ -451,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const float sl2 = p.scale_log2;
         const float resc_raw = kRescaleLog2 / sl2;  // threshold in raw score units
         float m_run = -INFINITY;  // reference max (raw units)
-        float l_run = 0.f;        // this half's share of the row sum
+        uint64_t l2x = 0ull;      // row sum, two partial sums in one register pair
         bool ok = true;
         const int W = p.window;
         for (int j = 0; j < n_kv; ++j) {
@@ -459,19 +443,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], j & 1, abort_flag, p.status, limit));
             if (!ok) break;
             tc_fence_after();
-            uint32_t sr[2][32];
-            tmem_ld32(tS, sr[0]);
-            tmem_ld32(tS + 32, sr[1]);
-            tmem_wait_ld(sr[0]);
-            tmem_wait_ld(sr[1]);
-            const int kbase = w.kv_lo + j * kTileN + 64 * half;  // position of this half's first key
-            const bool need_mask = (kbase + 63 > w.min_pos) || (MODE == kModeLocal && kbase < w.max_pos - W + 1);
+            uint32_t sr[4][32];
+            #pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sr[c]);
+            #pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_wait_ld(sr[c]);
+            const int kbase = w.kv_lo + j * kTileN;  // position of the tile's first key
+            const bool need_mask = (kbase + kTileN - 1 > w.min_pos) || (MODE == kModeLocal && kbase < w.max_pos - W + 1);
             if (need_mask) {
                 const int hi = pos - kbase;                                          // keep column c <= hi
                 const int lo = (MODE == kModeLocal) ? pos - W + 1 - kbase : INT_MIN;  // keep column c >= lo
                 // Selects, not branches: a per-element branch costs more than the exponentials.
                 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
+                for (int c = 0; c < 4; ++c) {
                     #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int col = c * 32 + e;
@@ -481,113 +465,88 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             }
             float mx[4];
             #pragma unroll
-            for (int t = 0; t < 4; ++t)
-                mx[t] = fmaxf(__uint_as_float(sr[t >> 1][(t & 1) * 16]), __uint_as_float(sr[t >> 1][(t & 1) * 16 + 1]));
-            #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const uint32_t* rr = &sr[t >> 1][(t & 1) * 16];
+            for (int c = 0; c < 4; ++c) {
+                mx[c] = fmaxf(__uint_as_float(sr[c][0]), __uint_as_float(sr[c][1]));
                 #pragma unroll
-                for (int e = 2; e < 16; e += 2) mx[t] = fmax3(mx[t], __uint_as_float(rr[e]), __uint_as_float(rr[e + 1]));
+                for (int e = 2; e < 32; e += 2) mx[c] = fmax3(mx[c], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
             }
-            const float m_half = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
-            // Combine with the other half of the row.  The other half also read its S
-            // columns before arriving here, so P may overwrite them after this point.
-            xch[half * 128 + r] = m_half;
-            mbar_arrive(pair);
-            ok = __all_sync(0xffffffffu, mbar_wait(pair, j & 1, abort_flag, p.status, limit));
-            if (!ok) break;
-            const float mt = fmaxf(m_half, xch[(half ^ 1) * 128 + r]);
+            const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             const float m_new = fmaxf(m_run, mt);
-            const bool need = m_new > m_run + resc_raw;  // the same decision in both halves
+            const bool need = m_new > m_run + resc_raw;
             float alpha = 1.f;
             if (need) {
                 alpha = (m_run == -INFINITY) ? 0.f : fast_exp2((m_run - m_new) * sl2);
                 m_run = m_new;
-                l_run *= alpha;
+                l2x = f2_mul(l2x, f2_pack(alpha, alpha));
             }
             const float mref = (m_run == -INFINITY) ? 0.f : m_run * sl2;
-            __syncwarp();
             // Paired fp32 instructions for the scaling and the row sums.
             const uint64_t sl2x2 = f2_pack(sl2, sl2), nmref2 = f2_pack(-mref, -mref);
-            uint64_t ls2[2] = {0ull, 0ull};
             #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 uint32_t pk[16];
                 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    const int col = 64 * half + c * 32 + e;
                     float x0, x1, p0, p1;
                     f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), sl2x2, nmref2),
                               x0, x1);
-                    // A share of the pairs may run on the FMA pipe to unload the MUFU unit.
-                    if (use_poly(col / 2)) {
-                        exp2_poly2(x0, x1, p0, p1);
-                    } else {
-                        p0 = fast_exp2(x0);
-                        p1 = fast_exp2(x1);
-                    }
-                    ls2[(e >> 1) & 1] = f2_add(ls2[(e >> 1) & 1], f2_pack(p0, p1));
+                    p0 = fast_exp2(x0);
+                    p1 = fast_exp2(x1);
+                    l2x = f2_add(l2x, f2_pack(p0, p1));
                     pk[e / 2] = pack_bf16x2(p0, p1);
                 }
-                tmem_st16(tP + c * 16, pk);
-            }
-            {
-                const uint64_t lsum = f2_add(ls2[0], ls2[1]);
-                float l0, l1;
-                f2_unpack(lsum, l0, l1);
-                l_run += l0 + l1;
-            }
-            // Rare: the row maximum grew past the threshold, so O must be rescaled
-            // before any PV of this tile (PV of tile j-1 is complete: see header).
-            // The first half rescales all D columns of the row: the first P part's
-            // MMAs (issued as soon as this half has arrived) write every column of
-            // O, so the second half must not touch O while they may run.  Both
-            // halves took the same decision and hold the same alpha.
-            const bool any = __any_sync(0xffffffffu, need);  // also reconverges the warp
-            if (any && j > 0 && half == 0) {
-                #pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t orr[32];
-                    tmem_ld32(tO_row + c * 32, orr);
-                    tmem_wait_ld(orr);
-                    #pragma unroll
-                    for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-                    tmem_st32(tO_row + c * 32, orr);
+                tmem_st16(tS + c * 16, pk);
+                if (c == 1) {
+                    // Rare: the row maximum grew past the threshold, so O must be rescaled
+                    // before any PV of this tile (PV of tile j-1 is complete: the commit
+                    // that signalled S(j) covers it).  The PV MMAs of the first P part
+                    // write every column of O, so this comes before that part is published.
+                    const bool any = __any_sync(0xffffffffu, need);  // also reconverges the warp
+                    if (any && j > 0) {
+                        #pragma unroll 1
+                        for (int cc = 0; cc < D / 32; ++cc) {
+                            uint32_t orr[32];
+                            tmem_ld32(tO + cc * 32, orr);
+                            tmem_wait_ld(orr);
+                            #pragma unroll
+                            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                            tmem_st32(tO + cc * 32, orr);
+                        }
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(&p_full[kPParts * wg + 0]);
                 }
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&p_full[2 * wg + half]);
+            mbar_arrive(&p_full[kPParts * wg + 1]);
         }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, abort_flag, p.status, limit));
         if (ok) {
-            // Row sum: the two halves' shares.
-            xch[half * 128 + r] = l_run;
-            mbar_arrive(pair);
-            ok = __all_sync(0xffffffffu, mbar_wait(pair, n_kv & 1, abort_flag, p.status, limit));
-        }
-        if (ok) {
             tc_fence_after();
-            const float l_row = l_run + xch[(half ^ 1) * 128 + r];
+            float l_lo, l_hi;
+            f2_unpack(l2x, l_lo, l_hi);
+            const float l_row = l_lo + l_hi;
             const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
-            uint16_t* orow = p.out + ((size_t)zq * p.L + w.s0 + pos) * D + (D / 2) * half;
+            uint16_t* orow = p.out + ((size_t)zq * p.L + w.s0 + pos) * D;
             // Saved for the backward pass: the row's log-sum-exp (exp2 domain) and,
             // for selected rows, the global branch before the gate.
             const size_t srow = MODE == kModeGlobal ? (size_t)head * p.sel_stride + w.sel_base + my_row0 + r : 0;
-            if (p.lse && row_valid && half == 0) {
+            if (p.lse && row_valid) {
                 const float lse2 = l_row > 0.f ? m_run * sl2 + log2f(l_row) : INFINITY;
                 if (MODE == kModeLocal) p.lse[(size_t)zq * p.L + w.s0 + pos] = lse2;
                 else p.lse[srow] = lse2;
             }
-            uint16_t* grow = (MODE == kModeGlobal && p.glob) ? p.glob + srow * D + (D / 2) * half : nullptr;
-            uint16_t* lrow = (MODE == kModeGlobal && p.loc_sel) ? p.loc_sel + srow * D + (D / 2) * half : nullptr;
+            uint16_t* grow = (MODE == kModeGlobal && p.glob) ? p.glob + srow * D : nullptr;
+            uint16_t* lrow = (MODE == kModeGlobal && p.loc_sel) ? p.loc_sel + srow * D : nullptr;
             float gsig = 0.f;
             if (MODE == kModeGlobal && p.merge && row_valid) {
                 const float g = p.gate[(size_t)w.b * p.L + w.s0 + pos];
                 gsig = 1.f / (1.f + expf(-g));
             }
             #pragma unroll 1
-            for (int c = 0; c < D / 64; ++c) {
+            for (int c = 0; c < D / 32; ++c) {
                 uint32_t orr[32];
                 __syncwarp();
                 tmem_ld32(tO + c * 32, orr);
@@ -650,6 +609,18 @@ cudaError_t launch_one(const AttnParams& p, dim3 grid, cudaStream_t stream)
 {
     const size_t smem = Geometry<D>::kBytes + 1024;
     auto kern = attn_fwd_kernel<D, MODE>;
+    // The register split (setmaxnreg) hands out exactly what the launch holds; a build
+    // whose kernel was given fewer registers per thread would make the increase wait
+    // forever, so it is refused here instead of launched.
+    static const cudaError_t regs_ok = [&] {
+        cudaFuncAttributes fa;
+        cudaError_t r = cudaFuncGetAttributes(&fa, kern);
+        if (r != cudaSuccess) return r;
+        return (long)fa.numRegs * kThreads >= 128L * kProducerRegs + 128L * kNumQ * kSoftmaxRegs
+                   ? cudaSuccess
+                   : cudaErrorInvalidConfiguration;
+    }();
+    if (regs_ok != cudaSuccess) return regs_ok;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, kThreads, smem, stream>>>(p);
@@ -705,3 +676,4 @@ cudaError_t launch_timeout_probe(uint32_t* status, unsigned long long limit_ns, 
 }
 
 }  // namespace logo
+

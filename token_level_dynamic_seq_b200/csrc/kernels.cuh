@@ -39,7 +39,14 @@ __host__ __device__ inline int64_t budget_count(double ratio, int64_t len)
 constexpr int kTileM = 128;   // query rows per Q tile (= TMEM lanes)
 constexpr int kTileN = 128;   // keys per K/V tile
 constexpr int kNumQ = 2;      // Q tiles per CTA, one softmax warpgroup each
-constexpr int kThreads = 64 + 256 * kNumQ;  // TMA warp, MMA warp, two warpgroups per query tile
+constexpr int kThreads = 128 + 128 * kNumQ;  // producer warpgroup (TMA, MMA, 2 idle), one warpgroup per query tile
+// Registers per thread after the producer warpgroup hands its share to the softmax
+// warpgroups (setmaxnreg).  The launch holds kThreads * 168 (the compiler's count
+// under __launch_bounds__(kThreads, 1)); the split must not exceed it, or the
+// increase would wait for registers that never come free.
+constexpr int kProducerRegs = 56;
+constexpr int kSoftmaxRegs = 224;
+static_assert(128 * kProducerRegs + 128 * kNumQ * kSoftmaxRegs <= kThreads * 168, "register split above the launch total");
 
 enum AttnMode : int { kModeLocal = 0, kModeGlobal = 1 };
 

@@ -90,6 +90,21 @@ LOGO_DEVICE_INLINE bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* 
     }
 }
 
+// ---------------------------------------------------------------- register split
+
+// Warpgroup-wide: lower (dealloc) or raise (alloc) this warpgroup's registers per thread.
+template <uint32_t N>
+LOGO_DEVICE_INLINE void reg_dealloc()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+
+template <uint32_t N>
+LOGO_DEVICE_INLINE void reg_alloc()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- TMA
 
 LOGO_DEVICE_INLINE void tma_prefetch_desc(const CUtensorMap* map)
@@ -271,25 +286,6 @@ LOGO_DEVICE_INLINE float fmax3(float a, float b, float c)
     return y;
 }
 
-// 2^x for x <= 8 on the FMA pipe (no MUFU): x = n + f with n = round(x),
-// f in [-1/2, 1/2] (rounding by adding and subtracting 1.5 * 2^23), then
-// 2^x = 2^n * p(f) with p the degree-3 minimax polynomial for the relative
-// error of 2^f on [-1/2, 1/2] (max relative error 7.5e-5, derived by
-// gen_exp2_poly.py with the Remez exchange), and 2^n applied by adding n to
-// the exponent field.  x is clamped at -125 so the result stays a normal
-// number (2^-125 is far below anything that survives the bf16 P tile).
-LOGO_DEVICE_INLINE float exp2_poly(float x)
-{
-    x = fmaxf(x, -125.0f);
-    const float t = __fadd_rn(x, 12582912.0f);      // round(x) in the low mantissa bits
-    const float n = __fadd_rn(t, -12582912.0f);
-    const float f = __fadd_rn(x, -n);
-    float p = fmaf(__uint_as_float(0x3d61fbb0u), f, __uint_as_float(0x3e786f0du));
-    p = fmaf(p, f, __uint_as_float(0x3f31798du));
-    p = fmaf(p, f, __uint_as_float(0x3f7ffb49u));
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 // Paired fp32 arithmetic (one instruction for two lanes of a 64-bit register
 // pair; sm_100 and later).  f2 values hold {lo, hi}.
 LOGO_DEVICE_INLINE uint64_t f2_pack(float lo, float hi)
@@ -330,26 +326,6 @@ LOGO_DEVICE_INLINE uint64_t f2_mul(uint64_t a, uint64_t b)
     uint64_t d;
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
-}
-
-// exp2_poly on a pair, with the additions and the polynomial in paired
-// instructions: the same arithmetic and result bits as exp2_poly per lane.
-LOGO_DEVICE_INLINE void exp2_poly2(float x0, float x1, float& y0, float& y1)
-{
-    const uint64_t x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-    const uint64_t t = f2_add(x, f2_pack(12582912.0f, 12582912.0f));
-    const uint64_t n = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
-    const uint64_t f = f2_sub(x, n);
-    const float c3 = __uint_as_float(0x3d61fbb0u), c2 = __uint_as_float(0x3e786f0du);
-    const float c1 = __uint_as_float(0x3f31798du), c0 = __uint_as_float(0x3f7ffb49u);
-    uint64_t p = f2_fma(f2_pack(c3, c3), f, f2_pack(c2, c2));
-    p = f2_fma(p, f, f2_pack(c1, c1));
-    p = f2_fma(p, f, f2_pack(c0, c0));
-    float p0, p1, t0, t1;
-    f2_unpack(p, p0, p1);
-    f2_unpack(t, t0, t1);
-    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 LOGO_DEVICE_INLINE uint32_t pack_bf16x2(float lo, float hi)
