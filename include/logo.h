@@ -70,7 +70,9 @@ typedef enum {
     LOGO_ERR_WORKSPACE = 3,      /* workspace missing or smaller than logo_workspace_size() */
     LOGO_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed (see logo_last_error) */
     LOGO_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait ran out (read by logo_check) */
-    LOGO_ERR_CAPACITY = 6        /* more tokens passed a threshold than the output holds (read by logo_check) */
+    LOGO_ERR_CAPACITY = 6,       /* more tokens passed a threshold than the output holds (read by logo_check) */
+    LOGO_ERR_BOUNDS = 7          /* debug build (LOGO_DEBUG_BOUNDS) only: a kernel's index check failed and
+                                    the access was skipped (read by logo_check) */
 } logo_status;
 
 /* Raw bf16 bit pattern. */
@@ -386,6 +388,12 @@ LOGO_API const char *logo_status_string(logo_status status);
 
 /* Details of the last error raised on the calling host thread ("" if none). */
 LOGO_API const char *logo_last_error(void);
+
+/* How this library was built: bit 0 (LOGO_BUILD_DEBUG_BOUNDS) is set in the
+ * debug build whose kernels check every TMA coordinate, gathered row and
+ * stored row before the access (make debug: liblogo_debug.so). */
+#define LOGO_BUILD_DEBUG_BOUNDS 1u
+LOGO_API unsigned logo_build_flags(void);
 
 #ifdef __cplusplus
 }

@@ -32,7 +32,7 @@ def declared_symbols():
 def test_library_exports_every_declared_symbol():
     lib = logo.load_library()
     names = declared_symbols()
-    assert len(names) == 21, names
+    assert len(names) == 22, names
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(logo.EXPORTED)

@@ -29,14 +29,15 @@ CSRC = os.path.join(_HERE, "csrc")
 
 LOGO_OK = 0
 _STATUS = {0: "LOGO_OK", 1: "LOGO_ERR_INVALID_ARG", 2: "LOGO_ERR_UNSUPPORTED", 3: "LOGO_ERR_WORKSPACE",
-           4: "LOGO_ERR_CUDA", 5: "LOGO_ERR_DEVICE_TIMEOUT", 6: "LOGO_ERR_CAPACITY"}
+           4: "LOGO_ERR_CUDA", 5: "LOGO_ERR_DEVICE_TIMEOUT", 6: "LOGO_ERR_CAPACITY",
+           7: "LOGO_ERR_BOUNDS"}
 
 EXPORTED = ("logo_num_selected", "logo_workspace_size", "logo_workspace_init", "logo_select",
             "logo_local_attn", "logo_global_attn_sparse", "logo_forward", "logo_check",
             "logo_selftest_timeout", "logo_status_string", "logo_last_error",
             "logo_global_attn_sparse_noalloc", "logo_select_threshold", "logo_threshold_update",
             "logo_decode_workspace_size", "logo_decode", "logo_forward_train", "logo_backward_workspace_size",
-            "logo_backward", "logo_forward_host_buffer_size", "logo_forward_host")
+            "logo_backward", "logo_forward_host_buffer_size", "logo_forward_host", "logo_build_flags")
 
 
 class LogoError(RuntimeError):
@@ -81,6 +82,7 @@ def load_library(path: str | None = None):
             "logo_selftest_timeout": ([vp, sz, ctypes.c_uint, vp], i32),
             "logo_status_string": ([i32], ctypes.c_char_p),
             "logo_last_error": ([], ctypes.c_char_p),
+            "logo_build_flags": ([], ctypes.c_uint),
             "logo_global_attn_sparse_noalloc": ([vp, vp, vp, vp, vp, vp, sp, i32, flt, i32, vp, vp], i32),
             "logo_select_threshold": ([vp, sp, vp, i32, vp, vp, vp, sz, vp], i32),
             "logo_threshold_update": ([vp, sp, dbl, flt, vp, vp, vp, sz, vp], i32),

@@ -762,6 +762,8 @@ logo_status logo_check(const void* ws, logo_stream_t stream)
         return fail(LOGO_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait ran out (status 0x%x)", status);
     if (status & logo::kStatusBadArgument)
         return fail(LOGO_ERR_INVALID_ARG, "a kernel met an argument it cannot handle (status 0x%x)", status);
+    if (status & logo::kStatusBounds)
+        return fail(LOGO_ERR_BOUNDS, "a debug bounds check failed and skipped an access (status 0x%x)", status);
     if (status & logo::kStatusCapacity)
         return fail(LOGO_ERR_CAPACITY, "more tokens passed the threshold than max_selected (status 0x%x)", status);
     return LOGO_OK;
@@ -893,10 +895,20 @@ const char* logo_status_string(logo_status s)
         case LOGO_ERR_CUDA: return "LOGO_ERR_CUDA";
         case LOGO_ERR_DEVICE_TIMEOUT: return "LOGO_ERR_DEVICE_TIMEOUT";
         case LOGO_ERR_CAPACITY: return "LOGO_ERR_CAPACITY";
+        case LOGO_ERR_BOUNDS: return "LOGO_ERR_BOUNDS";
     }
     return "LOGO_ERR_UNKNOWN";
 }
 
 const char* logo_last_error(void) { return g_last_error; }
+
+unsigned logo_build_flags(void)
+{
+#ifdef LOGO_DEBUG_BOUNDS
+    return LOGO_BUILD_DEBUG_BOUNDS;
+#else
+    return 0u;
+#endif
+}
 
 }  // extern "C"

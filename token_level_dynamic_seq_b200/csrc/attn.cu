@@ -18,7 +18,7 @@
 // shared memory by TMA and feeds both query tiles.
 //
 // Warp roles (12 warps, three warpgroups):
-//   warp 0       TMA producer: Q tiles (local mode) and the K/V ring.
+//   warp 0       TMA producer: Q tiles (local mode) and the K/V slots.
 //   warp 1       tcgen05 issuer (one thread): S_i = Q_i K^T into TMEM, then
 //                O_i += P_i V with P_i read straight from TMEM.
 //   warps 2-3    idle; with warps 0-1 they form the producer warpgroup, which
@@ -39,10 +39,12 @@
 //   PV_i(j), S_i(j+1).  S_i(j+1) overwrites the TMEM columns of P_i(j) only
 //   after PV_i(j) has read them, because tcgen05 MMAs from one thread execute
 //   in issue order; and the commit that signals S_i(j+1) also covers
-//   PV_i(j), so O_i may be rescaled as soon as S_i(j+1) is seen.  P_i(j) is
-//   published in two parts (keys 0-63, then 64-127) and the MMAs of the first
-//   part write all of O_i, so a rescale of O_i happens before the first part
-//   is published.
+//   PV_i(j), so O_i may be rescaled as soon as S_i(j+1) is seen, and is, before
+//   P_i(j) is published.
+// The MMA-issuing thread is the pipe's bottleneck (it reaches every P barrier
+// after the softmax has completed it), so it waits on as few barriers as the
+// data flow allows: one per key/value pair (K(j+1) and V(j) travel together),
+// one per published P.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -57,12 +59,13 @@ namespace logo {
 
 namespace {
 
-constexpr int kKStages = 2;
-constexpr int kVStages = 2;
+// K/V staging: two slots of one K tile and one V tile each.  Slot j % 2 receives the
+// pair (K(j+1), V(j)) in one transaction: PV(j) and S(j+1) are issued in the same
+// step, so the two tiles are needed together.  K(0) goes alone into slot 1 first.
+constexpr int kSlots = 2;
+constexpr int kKStages = kSlots;
+constexpr int kVStages = kSlots;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
-// P_i is published in two column blocks (keys 0-63, then 64-127): the PV MMAs of
-// the first start while the softmax computes the second.
-constexpr int kPParts = 2;
 
 template <int D>
 struct Geometry {
@@ -74,7 +77,7 @@ struct Geometry {
     static constexpr int kKOff = kQOff + kNumQ * kQBytes;
     static constexpr int kVOff = kKOff + kKStages * kKVBytes;
     static constexpr int kBarOff = kVOff + kVStages * kKVBytes;
-    static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + (1 + kPParts) * kNumQ + 2;
+    static constexpr int kNumBars = 1 + 2 * kSlots + 2 * kNumQ + 2;
     static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
     static constexpr int kTmemS = 0;          // S_i at column 128 * i
     static constexpr int kTmemO = 128 * kNumQ; // O_i at column 256 + D * i
@@ -98,6 +101,25 @@ struct Work {
 };
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Debug build (-DLOGO_DEBUG_BOUNDS): every TMA coordinate, gathered row and stored
+// row is checked against the tensor it addresses before the access.  A failed check
+// sets kStatusBounds, raises the CTA's abort flag (so every wait of the CTA gives up at
+// once) and the access is skipped.  In the normal build the checks compile away.
+__device__ __forceinline__ bool in_bounds(bool ok, uint32_t* status, volatile int* abort_flag)
+{
+#ifdef LOGO_DEBUG_BOUNDS
+    if (!ok) {
+        atomicOr(status, kStatusBounds);
+        *abort_flag = 1;
+    }
+    return ok;
+#else
+    (void)status;
+    (void)abort_flag;
+    return true;
+#endif
+}
 
 template <int MODE>
 __device__ Work make_work(const AttnParams& p)
@@ -207,13 +229,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     uint8_t* sV = smem + Geo::kVOff;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Geo::kBarOff);
     uint64_t* q_full = bars;
-    uint64_t* k_full = q_full + 1;
-    uint64_t* k_empty = k_full + kKStages;
-    uint64_t* v_full = k_empty + kKStages;
-    uint64_t* v_empty = v_full + kVStages;
-    uint64_t* s_full = v_empty + kVStages;
-    uint64_t* p_full = s_full + kNumQ;        // [kNumQ][kPParts]: part k of P_i written
-    uint64_t* o_full = p_full + kPParts * kNumQ;
+    uint64_t* kv_full = q_full + 1;           // [kSlots]: the slot's tiles have landed
+    uint64_t* kv_empty = kv_full + kSlots;    // [kSlots]: the MMAs that read the slot have completed
+    uint64_t* s_full = kv_empty + kSlots;
+    uint64_t* p_full = s_full + kNumQ;        // [kNumQ]: P_i written
+    uint64_t* o_full = p_full + kNumQ;
     uint64_t* drain = o_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -233,16 +253,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, MODE == kModeLocal ? 1 : 128 * kNumQ);
-        for (int s = 0; s < kKStages; ++s) {
-            mbar_init(&k_full[s], 1);
-            mbar_init(&k_empty[s], 1);
-        }
-        for (int s = 0; s < kVStages; ++s) {
-            mbar_init(&v_full[s], 1);
-            mbar_init(&v_empty[s], 1);
+        for (int s = 0; s < kSlots; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
         }
         for (int i = 0; i < kNumQ; ++i) mbar_init(&s_full[i], 1);
-        for (int i = 0; i < kPParts * kNumQ; ++i) mbar_init(&p_full[i], 128);
+        for (int i = 0; i < kNumQ; ++i) mbar_init(&p_full[i], 128);
         mbar_init(o_full, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -270,8 +286,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             tma_prefetch_desc(&p.tm_k);
             tma_prefetch_desc(&p.tm_v);
             const uint64_t pol_kv = policy_evict_last();
-            bool ok = true;
-            if (MODE == kModeLocal) {
+            const int slabs = p.cu_seqlens ? 1 : p.nseq;  // batch rows of the tensors
+            bool ok = in_bounds(zkv >= 0 && zkv < slabs * p.Hkv, p.status, abort_flag);
+            // A tile with no rows (the second tile past a sequence's end) is still loaded:
+            // its rows past the tensor's end read as zeros.
+            for (int i = 0; i < kNumQ && ok && MODE == kModeLocal; ++i)
+                ok = in_bounds(w.nrows[i] <= 0 || (w.s0 + w.row0[i] >= 0 && w.s0 + w.row0[i] < p.L &&
+                                                   w.b * p.Hq + w.head[i] >= 0 && w.b * p.Hq + w.head[i] < slabs * p.Hq),
+                               p.status, abort_flag);
+            bool q_armed = false;
+            if (MODE == kModeLocal && ok) {
+                q_armed = true;
                 tma_prefetch_desc(&p.tm_q);
                 const uint64_t pol_q = policy_evict_first();
                 mbar_arrive_expect_tx(q_full, kNumQ * Geo::kQBytes);
@@ -280,36 +305,45 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                         tma_load_3d(sQ + i * Geo::kQBytes + c * Geo::kChunkBytes, &p.tm_q, q_full, c * 64,
                                     w.s0 + w.row0[i], w.b * p.Hq + w.head[i], pol_q);
             }
-            int k_armed[kKStages], v_armed[kVStages];
-            for (int s = 0; s < kKStages; ++s) k_armed[s] = 0;
-            for (int s = 0; s < kVStages; ++s) v_armed[s] = 0;
+            // Transactions on slot s: use n of the slot (n = 0, 1, ...) completes phase n of
+            // kv_full[s]; slot 1's use 0 is K(0) alone, then pair j sits in slot j % 2 as
+            // that slot's use (j + (j & 1)) / 2.
+            int armed[kSlots] = {0, 0};
+            auto slot_use = [](int j) { return (j + (j & 1)) / 2; };
+            if (ok) ok = in_bounds(w.s0 + w.kv_lo >= 0 && w.s0 + w.kv_lo < p.L, p.status, abort_flag);
+            if (ok) {
+                mbar_arrive_expect_tx(&kv_full[1], Geo::kKVBytes);
+                ++armed[1];
+                for (int c = 0; c < Geo::kChunks; ++c)
+                    tma_load_3d(sK + 1 * Geo::kKVBytes + c * Geo::kChunkBytes, &p.tm_k, &kv_full[1], c * 64,
+                                w.s0 + w.kv_lo, zkv, pol_kv);
+            }
             for (int j = 0; j < n_kv && ok; ++j) {
-                const int row = w.s0 + w.kv_lo + j * kTileN;
-                const int ks = j % kKStages;
-                if (j >= kKStages) ok = mbar_wait(&k_empty[ks], ((j / kKStages) - 1) & 1, abort_flag, p.status, limit);
+                const int sl = j & 1;
+                const int use = slot_use(j);
+                const bool with_k = j + 1 < n_kv;
+                const int row_v = w.s0 + w.kv_lo + j * kTileN;
+                const int row_k = row_v + kTileN;
+                if (!in_bounds(row_v >= 0 && row_v < p.L && (!with_k || row_k < p.L), p.status, abort_flag)) break;
+                // the slot's previous contents have been read
+                if (use >= 1) ok = mbar_wait(&kv_empty[sl], (use - 1) & 1, abort_flag, p.status, limit);
                 if (!ok) break;
-                mbar_arrive_expect_tx(&k_full[ks], Geo::kKVBytes);
-                ++k_armed[ks];
+                mbar_arrive_expect_tx(&kv_full[sl], (with_k ? 2 : 1) * Geo::kKVBytes);
+                ++armed[sl];
                 for (int c = 0; c < Geo::kChunks; ++c)
-                    tma_load_3d(sK + ks * Geo::kKVBytes + c * Geo::kChunkBytes, &p.tm_k, &k_full[ks], c * 64, row,
+                    tma_load_3d(sV + sl * Geo::kKVBytes + c * Geo::kChunkBytes, &p.tm_v, &kv_full[sl], c * 64, row_v,
                                 zkv, pol_kv);
-                const int vs = j % kVStages;
-                if (j >= kVStages) ok = mbar_wait(&v_empty[vs], ((j / kVStages) - 1) & 1, abort_flag, p.status, limit);
-                if (!ok) break;
-                mbar_arrive_expect_tx(&v_full[vs], Geo::kKVBytes);
-                ++v_armed[vs];
-                for (int c = 0; c < Geo::kChunks; ++c)
-                    tma_load_3d(sV + vs * Geo::kKVBytes + c * Geo::kChunkBytes, &p.tm_v, &v_full[vs], c * 64, row,
-                                zkv, pol_kv);
+                if (with_k)
+                    for (int c = 0; c < Geo::kChunks; ++c)
+                        tma_load_3d(sK + sl * Geo::kKVBytes + c * Geo::kChunkBytes, &p.tm_k, &kv_full[sl], c * 64,
+                                    row_k, zkv, pol_kv);
             }
             if (*abort_flag) {
                 // Let every copy this thread started land before the CTA exits.
                 volatile int dummy = 0;
-                for (int s = 0; s < kKStages; ++s)
-                    if (k_armed[s]) mbar_wait(&k_full[s], (k_armed[s] - 1) & 1, &dummy, nullptr, limit);
-                for (int s = 0; s < kVStages; ++s)
-                    if (v_armed[s]) mbar_wait(&v_full[s], (v_armed[s] - 1) & 1, &dummy, nullptr, limit);
-                if (MODE == kModeLocal) mbar_wait(q_full, 0, &dummy, nullptr, limit);
+                for (int s2 = 0; s2 < kSlots; ++s2)
+                    if (armed[s2]) mbar_wait(&kv_full[s2], (armed[s2] - 1) & 1, &dummy, nullptr, limit);
+                if (q_armed) mbar_wait(q_full, 0, &dummy, nullptr, limit);
             }
         }
     } else if (warp == 1) {
@@ -328,52 +362,45 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     umma_ss(d_tmem, a, b, idesc_qk, kk > 0 ? 1u : 0u);
                 }
             };
-            // O_i += P_i V over the keys of P part `part` (128 / kPParts keys).
-            auto issue_pv = [&](int i, int vs, bool first, int part) {
+            // O_i += P_i V over the 128 keys of the tile.
+            auto issue_pv = [&](int i, int vs, bool first) {
                 const uint32_t d_tmem = tmem + Geo::kTmemO + D * i;
                 const uint32_t p_tmem = tmem + Geo::kTmemS + 128 * i;
-                constexpr int kSteps = 8 / kPParts;
                 #pragma unroll
-                for (int kk = kSteps * part; kk < kSteps * part + kSteps; ++kk) {
+                for (int kk = 0; kk < 8; ++kk) {
                     const uint64_t b = sdesc_sw128(sVa + vs * Geo::kKVBytes + kk * 2048, Geo::kChunkBytes, 1024);
                     umma_ts(d_tmem, p_tmem + kk * 8, b, idesc_pv, (!first || kk > 0) ? 1u : 0u);
                 }
             };
             bool ok = mbar_wait(q_full, 0, abort_flag, p.status, limit);
-            if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag, p.status, limit);
+            if (ok) ok = mbar_wait(&kv_full[1], 0, abort_flag, p.status, limit);  // K(0)
             if (ok) {
                 tc_fence_after();
                 for (int i = 0; i < kNumQ; ++i) {
-                    issue_s(i, 0);
+                    issue_s(i, 1);
                     umma_commit(&s_full[i]);
                 }
-                umma_commit(&k_empty[0]);
+                umma_commit(&kv_empty[1]);
             }
             for (int j = 0; j < n_kv && ok; ++j) {
                 const bool nxt = j + 1 < n_kv;
-                const int ks1 = (j + 1) % kKStages;
-                const int vs = j % kVStages;
-                if (nxt) ok = mbar_wait(&k_full[ks1], ((j + 1) / kKStages) & 1, abort_flag, p.status, limit);
-                if (ok) ok = mbar_wait(&v_full[vs], (j / kVStages) & 1, abort_flag, p.status, limit);
+                const int sl = j & 1;
+                // V(j) and, if there is one, K(j+1): the slot's use (j + (j & 1)) / 2
+                ok = mbar_wait(&kv_full[sl], ((j + (j & 1)) / 2) & 1, abort_flag, p.status, limit);
                 if (!ok) break;
                 tc_fence_after();
                 for (int i = 0; i < kNumQ && ok; ++i) {
-                    // P_i is published part by part while the softmax computes the rest.
-                    for (int part = 0; part < kPParts && ok; ++part) {
-                        ok = mbar_wait(&p_full[kPParts * i + part], j & 1, abort_flag, p.status, limit);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_pv(i, vs, j == 0, part);
-                    }
+                    ok = mbar_wait(&p_full[i], j & 1, abort_flag, p.status, limit);
                     if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(i, sl, j == 0);
                     if (nxt) {
-                        issue_s(i, ks1);
+                        issue_s(i, sl);
                         umma_commit(&s_full[i]);
                     }
                 }
                 if (!ok) break;
-                if (nxt) umma_commit(&k_empty[ks1]);
-                umma_commit(&v_empty[vs]);
+                umma_commit(&kv_empty[sl]);
             }
             if (ok) umma_commit(o_full);
             // Drain: everything issued above completes before TMEM is released.
@@ -419,6 +446,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     atomicOr(p.status, kStatusBadArgument);
                 }
             }
+            row_valid = row_valid && in_bounds(zq >= 0 && zq < (p.cu_seqlens ? 1 : p.nseq) * p.Hq && pos >= 0 &&
+                                                   pos < w.len && w.s0 + pos < p.L,
+                                               p.status, abort_flag);
             // Gather this row of Q into the 128B-swizzled tile.
             uint8_t* dst = sQ + wg * Geo::kQBytes;
             const int4* src = reinterpret_cast<const int4*>(p.q + ((size_t)zq * p.L + w.s0 + pos) * D);
@@ -496,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     pk[e / 2] = pack_bf16x2(p0, p1);
                 }
                 tmem_st16(tS + c * 16, pk);
-                if (c == 1) {
+                if (c == 3) {
                     // Rare: the row maximum grew past the threshold, so O must be rescaled
                     // before any PV of this tile (PV of tile j-1 is complete: the commit
                     // that signalled S(j) covers it).  The PV MMAs of the first P part
@@ -515,12 +545,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     }
                     tmem_wait_st();
                     tc_fence_before();
-                    mbar_arrive(&p_full[kPParts * wg + 0]);
+                    mbar_arrive(&p_full[wg]);
                 }
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&p_full[kPParts * wg + 1]);
         }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, abort_flag, p.status, limit));
         if (ok) {
@@ -530,6 +557,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             const float l_row = l_lo + l_hi;
             const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
             uint16_t* orow = p.out + ((size_t)zq * p.L + w.s0 + pos) * D;
+            if (row_valid)
+                row_valid = in_bounds(zq >= 0 && zq < (p.cu_seqlens ? 1 : p.nseq) * p.Hq && pos >= 0 && pos < w.len &&
+                                          w.s0 + pos < p.L,
+                                      p.status, abort_flag);
             // Saved for the backward pass: the row's log-sum-exp (exp2 domain) and,
             // for selected rows, the global branch before the gate.
             const size_t srow = MODE == kModeGlobal ? (size_t)head * p.sel_stride + w.sel_base + my_row0 + r : 0;

@@ -11,6 +11,7 @@ enum : uint32_t {
     kStatusTimeout = 1u,      // a bounded wait ran out
     kStatusBadArgument = 2u,  // a kernel met an argument it cannot handle
     kStatusCapacity = 4u,     // more tokens above the threshold than the output holds
+    kStatusBounds = 8u,       // debug build: an index check failed and the access was skipped
 };
 
 // Budget count, identical on host and device (see logo_num_selected in
