@@ -23,7 +23,7 @@
 //                O_i += P_i V with P_i read straight from TMEM.
 //   warps 2-3    idle; with warps 0-1 they form the producer warpgroup, which
 //                hands most of its registers to the softmax warpgroups
-//                (setmaxnreg: 56 registers per thread there, 224 in the softmax).
+//                (setmaxnreg: 88 registers per thread there, 208 in the softmax).
 //   warps 4-7    softmax for query tile 0: thread = row = TMEM lane, holding all
 //                128 scores of its row, so the row maximum is a thread-local
 //                reduction.
@@ -351,26 +351,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(kTileM, kTileN, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(kTileM, D, true);
-            const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+            // Descriptors of each operand's first slice, made once; the slice at byte offset
+            // `off` is the base plus off >> 4 (the start-address field is the low 14 bits and
+            // every shared-memory address here is below 2^18, so the sum never carries out).
+            const uint64_t dq0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+            const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+            const uint64_t dv0 = sdesc_sw128(smem_u32(sV), Geo::kChunkBytes, 1024);
             auto issue_s = [&](int i, int ks) {
                 const uint32_t d_tmem = tmem + Geo::kTmemS + 128 * i;
+                const uint64_t a0 = dq0 + (uint64_t)(i * (Geo::kQBytes >> 4));
+                const uint64_t b0 = dk0 + (uint64_t)(ks * (Geo::kKVBytes >> 4));
                 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * Geo::kChunkBytes + (kk & 3) * 32;
-                    const uint64_t a = sdesc_sw128(sQa + i * Geo::kQBytes + off, 16, 1024);
-                    const uint64_t b = sdesc_sw128(sKa + ks * Geo::kKVBytes + off, 16, 1024);
-                    umma_ss(d_tmem, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                    const uint64_t off = (uint64_t)((kk >> 2) * (Geo::kChunkBytes >> 4) + (kk & 3) * 2);
+                    umma_ss(d_tmem, a0 + off, b0 + off, idesc_qk, kk > 0 ? 1u : 0u);
                 }
             };
             // O_i += P_i V over the 128 keys of the tile.
             auto issue_pv = [&](int i, int vs, bool first) {
                 const uint32_t d_tmem = tmem + Geo::kTmemO + D * i;
                 const uint32_t p_tmem = tmem + Geo::kTmemS + 128 * i;
+                const uint64_t b0 = dv0 + (uint64_t)(vs * (Geo::kKVBytes >> 4));
                 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t b = sdesc_sw128(sVa + vs * Geo::kKVBytes + kk * 2048, Geo::kChunkBytes, 1024);
-                    umma_ts(d_tmem, p_tmem + kk * 8, b, idesc_pv, (!first || kk > 0) ? 1u : 0u);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ts(d_tmem, p_tmem + kk * 8, b0 + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
+                            (!first || kk > 0) ? 1u : 0u);
             };
             bool ok = mbar_wait(q_full, 0, abort_flag, p.status, limit);
             if (ok) ok = mbar_wait(&kv_full[1], 0, abort_flag, p.status, limit);  // K(0)

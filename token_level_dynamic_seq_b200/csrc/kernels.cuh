@@ -45,8 +45,8 @@ constexpr int kThreads = 128 + 128 * kNumQ;  // producer warpgroup (TMA, MMA, 2 
 // warpgroups (setmaxnreg).  The launch holds kThreads * 168 (the compiler's count
 // under __launch_bounds__(kThreads, 1)); the split must not exceed it, or the
 // increase would wait for registers that never come free.
-constexpr int kProducerRegs = 56;
-constexpr int kSoftmaxRegs = 224;
+constexpr int kProducerRegs = 88;
+constexpr int kSoftmaxRegs = 208;
 static_assert(128 * kProducerRegs + 128 * kNumQ * kSoftmaxRegs <= kThreads * 168, "register split above the launch total");
 
 enum AttnMode : int { kModeLocal = 0, kModeGlobal = 1 };
