@@ -366,20 +366,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, true);
             const uint32_t sQa = smem_u32(sQ), sDoa = smem_u32(sDo), sKa = smem_u32(sK), sVa = smem_u32(sV);
             // D[128 x 128] = A[128 x D] B[128 x D]^T, both K-major tiles.
+            // Each operand's descriptor is made once per call; the slice at byte offset `off`
+            // is that descriptor plus off >> 4 (the start-address field is the low 14 bits and
+            // every shared-memory address here is below 2^18, so the sum never carries out).
             auto issue_kmajor = [&](uint32_t d_tmem, uint32_t a_base, uint32_t b_base) {
+                const uint64_t a0 = sdesc_sw128(a_base, 16, 1024), b0 = sdesc_sw128(b_base, 16, 1024);
                 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * Geo::kChunkBytes + (kk & 3) * 32;
-                    umma_ss(d_tmem, sdesc_sw128(a_base + off, 16, 1024), sdesc_sw128(b_base + off, 16, 1024), idesc_s,
-                            kk > 0 ? 1u : 0u);
+                    const uint64_t off = (uint64_t)((kk >> 2) * (Geo::kChunkBytes >> 4) + (kk & 3) * 2);
+                    umma_ss(d_tmem, a0 + off, b0 + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
             // dQ += dS K: dS from TMEM (keys 0-63 in columns 0-31, keys 64-127 in 64-95).
             auto issue_dq = [&](int ks, bool first) {
+                const uint64_t b0 = sdesc_sw128(sKa + ks * Geo::kTile, Geo::kChunkBytes, 1024);
                 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t a = tmem + Geo::kTmemDP + (kk >> 2) * 64 + (kk & 3) * 8;
-                    const uint64_t b = sdesc_sw128(sKa + ks * Geo::kTile + kk * 2048, Geo::kChunkBytes, 1024);
+                    const uint64_t b = b0 + (uint64_t)(kk * (2048 >> 4));
                     umma_ts(tmem + Geo::kTmemDQ, a, b, idesc_dq, (!first || kk > 0) ? 1u : 0u);
                 }
             };
@@ -818,22 +822,26 @@ __global__ void __launch_bounds__(kKvThreads) bwd_dkdv_kernel(const __grid_const
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
             constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);
             const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV), sQa = smem_u32(sQ), sDoa = smem_u32(sDo);
+            // Each operand's descriptor is made once per call; the slice at byte offset `off`
+            // is that descriptor plus off >> 4 (the start-address field is the low 14 bits and
+            // every shared-memory address here is below 2^18, so the sum never carries out).
             auto issue_kmajor = [&](uint32_t d_tmem, uint32_t a_base, uint32_t b_base) {
+                const uint64_t a0 = sdesc_sw128(a_base, 16, 1024), b0 = sdesc_sw128(b_base, 16, 1024);
                 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * Geo::kChunkBytes + (kk & 3) * 32;
-                    umma_ss(d_tmem, sdesc_sw128(a_base + off, 16, 1024), sdesc_sw128(b_base + off, 16, 1024), idesc_s,
-                            kk > 0 ? 1u : 0u);
+                    const uint64_t off = (uint64_t)((kk >> 2) * (Geo::kChunkBytes >> 4) + (kk & 3) * 2);
+                    umma_ss(d_tmem, a0 + off, b0 + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
             // acc += X^T-tile (bf16 in the dP^T columns) times a [128 x D] tile.  Queries 32c .. 32c+31
             // of warpgroup h sit in columns 64h + 32c + which * 16 .. +15 (which 0: P^T, 1: dS^T).
             auto issue_acc = [&](uint32_t d_tmem, int which, uint32_t b_base, bool first) {
+                const uint64_t b0 = sdesc_sw128(b_base, Geo::kChunkBytes, 1024);
                 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t a = tmem + Geo::kTmemDP + (kk >> 2) * 64 + ((kk >> 1) & 1) * 32 + which * 16 +
                                        (kk & 1) * 8;
-                    const uint64_t bd = sdesc_sw128(b_base + kk * 2048, Geo::kChunkBytes, 1024);
+                    const uint64_t bd = b0 + (uint64_t)(kk * (2048 >> 4));
                     umma_ts(d_tmem, a, bd, idesc_acc, (!first || kk > 0) ? 1u : 0u);
                 }
             };
