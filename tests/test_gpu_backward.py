@@ -143,3 +143,22 @@ def test_backward_headline_one_group_in_full():
     close(dq[:, hs], ref["dq"], f"c32k group {hk} dq in full")
     close(dk[:, hk:hk + 1], ref["dk"], f"c32k group {hk} dk in full")
     close(dv[:, hk:hk + 1], ref["dv"], f"c32k group {hk} dv in full")
+
+
+def test_backward_varlen_one_group_in_full():
+    """The packed varlen workload (8 sequences, 67,706 tokens, W=2048, 25% global in clustered
+    bursts): every element of dQ, dK and dV of one key/value group against the oracle's
+    backward on that group alone (the selection is per sequence and depends on the gate only)."""
+    w = workloads.load("varlen")
+    gen = torch.Generator().manual_seed(11)
+    e = torch.randn(w.q.shape, generator=gen).bfloat16()
+    dq, dk, dv, _ = gpu_run(w, e)
+    G = w.Hq // w.Hkv
+    hk = 5
+    hs = slice(hk * G, (hk + 1) * G)
+    ref = oracle.backward(w.q[:, hs].contiguous(), w.k[:, hk:hk + 1].contiguous(), w.v[:, hk:hk + 1].contiguous(),
+                          w.g, e[:, hs].contiguous(), w.W, w.ratio, cu_seqlens=w.cu_seqlens)
+    T = int(w.cu_seqlens[-1])
+    close(dq[:, hs, :T], ref["dq"][:, :, :T], f"varlen group {hk} dq in full")
+    close(dk[:, hk:hk + 1, :T], ref["dk"][:, :, :T], f"varlen group {hk} dk in full")
+    close(dv[:, hk:hk + 1, :T], ref["dv"][:, :, :T], f"varlen group {hk} dv in full")

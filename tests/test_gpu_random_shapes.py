@@ -1,0 +1,79 @@
+"""Forward and backward on seeded random shapes, every element against the oracle.
+
+Each case draws its own shape from a seeded generator: batch or packed
+sequences (including empty and one-token ones), the query and key/value head
+counts (GQA groups of 1 to 5, odd and even), length (not a multiple of the
+128-row tile), head dimension 64 or 128, window (1, a few keys, or past the
+length) and ratio (0 to 1).  Selection must match bit for bit; outputs and
+gradients within the same tolerances as the fixed cases.
+"""
+import random
+
+import pytest
+import torch
+
+import oracle
+import token_level_dynamic_seq_b200 as logo
+from token_level_dynamic_seq_b200 import workloads
+
+from tests.test_gpu_parity import MAX_ABS, close, oracle_sel_lists, sel_lists, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def draw_case(seed):
+    rng = random.Random(1000 + seed)
+    Hkv = rng.choice([1, 2, 3])
+    G = rng.choice([1, 2, 3, 4, 5])
+    d = rng.choice([64, 128])
+    W = rng.choice([1, 2, 17, 128, 129, 300, 5000])
+    ratio = rng.choice([0.0, 0.05, 0.25, 0.5, 0.999, 1.0])
+    if rng.random() < 0.4:
+        seqlens = [rng.choice([0, 1, 2, 127, 128, 129, rng.randrange(3, 700)]) for _ in range(rng.randrange(1, 5))]
+        if sum(seqlens) == 0:
+            seqlens[0] = 5
+        B, L = 1, 0
+    else:
+        seqlens = None
+        B, L = rng.choice([1, 2]), rng.randrange(1, 800)
+    return B, Hkv * G, Hkv, L, d, W, ratio, seqlens
+
+
+CASES = list(range(12))
+
+
+@pytest.mark.parametrize("seed", CASES)
+def test_forward_random_shape(seed):
+    B, Hq, Hkv, L, d, W, ratio, lens = draw_case(seed)
+    w = workloads.make(B, Hq, Hkv, L, d, W, ratio, seed=seed, qkv_scale=1.0, seqlens=lens, name=f"random{seed}")
+    q, k, v, g, cu = to_dev(w)
+    ml = max(w.seqlens)
+    out, sel, cu_sel = logo.forward(q, k, v, g, w.W, w.ratio, cu_seqlens=cu, max_seqlen=ml if cu is not None else None)
+    torch.cuda.synchronize()
+    ref = oracle.forward(w.q, w.k, w.v, w.g, w.W, w.ratio, cu_seqlens=w.cu_seqlens)
+    assert sel_lists(sel, cu_sel) == oracle_sel_lists(w)
+    T = w.L if w.cu_seqlens is None else int(w.cu_seqlens[-1])
+    # Unscaled N(0,1) inputs with a short window give outputs up to |o| ~ 8, where one bf16
+    # rounding is up to 2^-6 and the merged row is rounded twice: the max-abs bound scales with
+    # the output as in the large-output tests, 2e-2 * max(1, max|ref| / 4); rel-L2 stays 5e-3.
+    r = ref["out"][:, :, :T]
+    close(out[:, :, :T], r, f"random {seed} {(B, Hq, Hkv, L, d, W, ratio, lens)}",
+          max_abs=MAX_ABS * max(1.0, r.abs().max().item() / 4.0))
+
+
+@pytest.mark.parametrize("seed", CASES[:6])
+def test_backward_random_shape(seed):
+    from tests.test_gpu_backward import close as close_grad, gpu_run
+
+    B, Hq, Hkv, L, d, W, ratio, lens = draw_case(seed)
+    w = workloads.make(B, Hq, Hkv, L, d, W, ratio, seed=seed, qkv_scale=1.0, seqlens=lens, name=f"random{seed}")
+    e = torch.randn(w.q.shape, generator=torch.Generator().manual_seed(seed)).bfloat16()
+    dq, dk, dv, dg = gpu_run(w, e)
+    ref = oracle.backward(w.q, w.k, w.v, w.g, e, w.W, w.ratio, cu_seqlens=w.cu_seqlens)
+    T = w.L if w.cu_seqlens is None else int(w.cu_seqlens[-1])
+    what = f"random {seed} {(B, Hq, Hkv, L, d, W, ratio, lens)}"
+    close_grad(dq[:, :, :T], ref["dq"][:, :, :T], what + " dq")
+    close_grad(dk[:, :, :T], ref["dk"][:, :, :T], what + " dk")
+    close_grad(dv[:, :, :T], ref["dv"][:, :, :T], what + " dv")
+    if (ref["dg"] != 0).any():
+        close_grad(dg[:, :T], ref["dg"][:, :T], what + " dgate")
