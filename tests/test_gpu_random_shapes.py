@@ -77,3 +77,27 @@ def test_backward_random_shape(seed):
     close_grad(dv[:, :, :T], ref["dv"][:, :, :T], what + " dv")
     if (ref["dg"] != 0).any():
         close_grad(dg[:, :T], ref["dg"][:, :T], what + " dgate")
+
+
+MEDIUM = [
+    # name, B, Hq, Hkv, L, d, W, ratio, seqlens: group sizes the named workloads do not use,
+    # at sizes that span many tiles (odd groups pair consecutive row tiles in one CTA)
+    ("odd group 3 varlen", 1, 6, 2, 0, 128, 700, 0.2, [3000, 1, 5000, 129]),
+    ("group 8", 1, 16, 2, 2500, 128, 1024, 0.25, None),
+    ("odd group 5 d64", 2, 5, 1, 1800, 64, 300, 0.3, None),
+]
+
+
+@pytest.mark.parametrize("case", MEDIUM, ids=[c[0] for c in MEDIUM])
+def test_forward_medium_edge_groups(case):
+    name, B, Hq, Hkv, L, d, W, ratio, lens = case
+    w = workloads.make(B, Hq, Hkv, L, d, W, ratio, seed=7, qkv_scale=1.0, seqlens=lens, name=name)
+    q, k, v, g, cu = to_dev(w)
+    ml = max(w.seqlens)
+    out, sel, cu_sel = logo.forward(q, k, v, g, w.W, w.ratio, cu_seqlens=cu, max_seqlen=ml if cu is not None else None)
+    torch.cuda.synchronize()
+    ref = oracle.forward(w.q, w.k, w.v, w.g, w.W, w.ratio, cu_seqlens=w.cu_seqlens)
+    assert sel_lists(sel, cu_sel) == oracle_sel_lists(w)
+    T = w.L if w.cu_seqlens is None else int(w.cu_seqlens[-1])
+    r = ref["out"][:, :, :T]
+    close(out[:, :, :T], r, name, max_abs=MAX_ABS * max(1.0, r.abs().max().item() / 4.0))
