@@ -216,7 +216,10 @@ __device__ DqWork dq_work(const BwdParams& p)
         w.len = p.L;
     }
     if (w.len <= 0) return w;
-    w.head = blockIdx.y;
+    // Local rows: x = row tile, y = head.  Selected rows: x = head, y = chunk, heaviest chunk
+    // first, so the longest prefixes of every head start in the first wave (chunk-fastest order
+    // left the last head's longest prefixes for the tail: 2.37 against 2.21 ms at 32K).
+    w.head = MODE == kModeLocal ? blockIdx.y : blockIdx.x;
     w.zq = w.b * p.Hq + w.head;
     if (MODE == kModeLocal) {
         w.row0 = blockIdx.x * 128;
@@ -233,7 +236,7 @@ __device__ DqWork dq_work(const BwdParams& p)
             if (threadIdx.x == 0) atomicOr(p.status, kStatusBadArgument);
             return w;
         }
-        const int c = ceil_div_i(k, 128) - 1 - (int)blockIdx.x;  // heaviest chunk first
+        const int c = ceil_div_i(k, 128) - 1 - (int)blockIdx.y;  // heaviest chunk first
         if (c < 0) return w;
         w.row0 = c * 128;
         w.nrows = min(128, k - w.row0);
@@ -1082,7 +1085,7 @@ cudaError_t launch_bwd_dq(int mode, int d, const BwdParams& p, int max_seqlen, c
 {
     dim3 grid;
     if (mode == kModeLocal) grid = dim3((max_seqlen + 127) / 128, p.Hq, p.nseq);
-    else grid = dim3((p.max_selected + 127) / 128, p.Hq, p.nseq);
+    else grid = dim3(p.Hq, (p.max_selected + 127) / 128, p.nseq);
     if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
     if (d == 64) {
         const size_t smem = DqGeo<64>::kBytes + 1024;
@@ -1096,6 +1099,8 @@ cudaError_t launch_bwd_dq(int mode, int d, const BwdParams& p, int max_seqlen, c
 
 cudaError_t launch_bwd_dkdv(int d, const BwdParams& p, int max_seqlen, cudaStream_t stream)
 {
+    // x = key tile, y = key/value head: the CTAs that run together share one head's Q and dout
+    // in L2 (head-fastest order balanced the tail no better and read 2.9x the DRAM bytes).
     const dim3 grid((max_seqlen + 127) / 128, p.Hkv, p.nseq);
     if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
     if (d == 64) return launch_big(bwd_dkdv_kernel<64>, KvGeo<64>::kBytes + 1024, grid, p, stream, kKvThreads);
