@@ -465,6 +465,28 @@ def test_timeout_is_reported_and_context_survives():
     close(out, ref["out"], "after timeout")
 
 
+def test_launch_after_timeout_does_no_work():
+    """Once a timeout is recorded in a workspace's status word, the attention launches that use
+    that workspace skip their work (a broken launch ends quickly): the output stays untouched
+    and the status still reports the timeout."""
+    w = workloads.load("c4k")
+    q, k, v, g, _ = to_dev(w)
+    sh = logo.make_shape(q, k)
+    ws = logo.workspace(sh, w.ratio, q.device)
+    sel_idx, cu_sel = logo.select(g, sh, w.ratio, ws)
+    torch.cuda.synchronize()
+    logo.selftest_timeout(ws, limit_us=2000)
+    sentinel = torch.full_like(q, 3.0)
+    out = sentinel.clone()
+    logo.local_attn(q, k, v, w.W, ws, out=out)
+    logo.global_attn_sparse(q, k, v, g, sel_idx, cu_sel, logo.num_selected(w.ratio, w.L), out, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out, sentinel)
+    with pytest.raises(logo.LogoError) as e:
+        logo.check(ws)
+    assert e.value.status == 5
+
+
 # --------------------------------------------------------------------------
 # caller-supplied selection lists that break the contract
 # --------------------------------------------------------------------------

@@ -241,16 +241,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // A CTA launched after another one recorded a timeout does no work, so a
-    // broken launch ends quickly instead of waiting out every CTA's limit.
-    __shared__ int sh_skip;
-    if (threadIdx.x == 0) sh_skip = (*reinterpret_cast<volatile uint32_t*>(p.status) & kStatusTimeout) ? 1 : 0;
-    __syncthreads();
-    if (sh_skip) return;
-
     const Work w = make_work<MODE>(p);
     if (!w.valid) return;  // uniform across the CTA
 
+    const int zkv = w.b * p.Hkv + w.hk;
+    // Producer state: thread 0 (the TMA lane) starts the first copies (the Q tiles, K(0)) right
+    // after it has initialised the barriers, before TMEM allocation and the CTA-wide sync.
+    bool p_ok = true, q_armed = false;
+    int armed[kSlots] = {0, 0};
+    // A CTA launched after another one recorded a timeout does no work past its first copies,
+    // so a broken launch ends quickly instead of waiting out every CTA's limit.  The status
+    // word is read while those copies are issued.
+    __shared__ int sh_skip;
     if (threadIdx.x == 0) {
         mbar_init(q_full, MODE == kModeLocal ? 1 : 128 * kNumQ);
         for (int s = 0; s < kSlots; ++s) {
@@ -263,6 +265,39 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
+        const uint32_t status0 = *reinterpret_cast<volatile uint32_t*>(p.status);
+        tma_prefetch_desc(&p.tm_k);
+        tma_prefetch_desc(&p.tm_v);
+        const int slabs = p.cu_seqlens ? 1 : p.nseq;  // batch rows of the tensors
+        p_ok = in_bounds(zkv >= 0 && zkv < slabs * p.Hkv, p.status, abort_flag);
+        // A tile with no rows (the second tile past a sequence's end) is still loaded:
+        // its rows past the tensor's end read as zeros.
+        for (int i = 0; i < kNumQ && p_ok && MODE == kModeLocal; ++i)
+            p_ok = in_bounds(w.nrows[i] <= 0 || (w.s0 + w.row0[i] >= 0 && w.s0 + w.row0[i] < p.L &&
+                                                 w.b * p.Hq + w.head[i] >= 0 && w.b * p.Hq + w.head[i] < slabs * p.Hq),
+                             p.status, abort_flag);
+        if (MODE == kModeLocal && p_ok) {
+            q_armed = true;
+            tma_prefetch_desc(&p.tm_q);
+            const uint64_t pol_q = policy_evict_first();
+            mbar_arrive_expect_tx(q_full, kNumQ * Geo::kQBytes);
+            for (int i = 0; i < kNumQ; ++i)
+                for (int c = 0; c < Geo::kChunks; ++c)
+                    tma_load_3d(sQ + i * Geo::kQBytes + c * Geo::kChunkBytes, &p.tm_q, q_full, c * 64,
+                                w.s0 + w.row0[i], w.b * p.Hq + w.head[i], pol_q);
+        }
+        // Transactions on slot s: use n of the slot (n = 0, 1, ...) completes phase n of
+        // kv_full[s]; slot 1's use 0 is K(0) alone, then pair j sits in slot j % 2 as
+        // that slot's use (j + (j & 1)) / 2.
+        if (p_ok) p_ok = in_bounds(w.s0 + w.kv_lo >= 0 && w.s0 + w.kv_lo < p.L, p.status, abort_flag);
+        if (p_ok) {
+            mbar_arrive_expect_tx(&kv_full[1], Geo::kKVBytes);
+            ++armed[1];
+            for (int c = 0; c < Geo::kChunks; ++c)
+                tma_load_3d(sK + 1 * Geo::kKVBytes + c * Geo::kChunkBytes, &p.tm_k, &kv_full[1], c * 64,
+                            w.s0 + w.kv_lo, zkv, policy_evict_last());
+        }
+        sh_skip = (status0 & kStatusTimeout) ? 1 : 0;
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, Geo::kTmemCols);
@@ -274,7 +309,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const uint32_t tmem = *tmem_slot;
     const uint64_t limit = p.timeout_ns;
     const int n_kv = w.n_kv;
-    const int zkv = w.b * p.Hkv + w.hk;
+    if (sh_skip) {
+        if (threadIdx.x == 0) {
+            // let the first copies land before the CTA exits
+            volatile int dummy = 0;
+            if (q_armed) mbar_wait(q_full, 0, &dummy, nullptr, limit);
+            if (armed[1]) mbar_wait(&kv_full[1], 0, &dummy, nullptr, limit);
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 1) {
+            tc_fence_after();
+            tmem_dealloc(tmem, Geo::kTmemCols);
+        }
+        return;
+    }
 
     if (warp < 4) {
       // Producer warpgroup: TMA (warp 0), tcgen05 issue (warp 1), two idle warps.
@@ -283,41 +332,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            tma_prefetch_desc(&p.tm_k);
-            tma_prefetch_desc(&p.tm_v);
+            // Q and K(0) are in flight (started before the CTA-wide sync); the pairs follow.
             const uint64_t pol_kv = policy_evict_last();
-            const int slabs = p.cu_seqlens ? 1 : p.nseq;  // batch rows of the tensors
-            bool ok = in_bounds(zkv >= 0 && zkv < slabs * p.Hkv, p.status, abort_flag);
-            // A tile with no rows (the second tile past a sequence's end) is still loaded:
-            // its rows past the tensor's end read as zeros.
-            for (int i = 0; i < kNumQ && ok && MODE == kModeLocal; ++i)
-                ok = in_bounds(w.nrows[i] <= 0 || (w.s0 + w.row0[i] >= 0 && w.s0 + w.row0[i] < p.L &&
-                                                   w.b * p.Hq + w.head[i] >= 0 && w.b * p.Hq + w.head[i] < slabs * p.Hq),
-                               p.status, abort_flag);
-            bool q_armed = false;
-            if (MODE == kModeLocal && ok) {
-                q_armed = true;
-                tma_prefetch_desc(&p.tm_q);
-                const uint64_t pol_q = policy_evict_first();
-                mbar_arrive_expect_tx(q_full, kNumQ * Geo::kQBytes);
-                for (int i = 0; i < kNumQ; ++i)
-                    for (int c = 0; c < Geo::kChunks; ++c)
-                        tma_load_3d(sQ + i * Geo::kQBytes + c * Geo::kChunkBytes, &p.tm_q, q_full, c * 64,
-                                    w.s0 + w.row0[i], w.b * p.Hq + w.head[i], pol_q);
-            }
-            // Transactions on slot s: use n of the slot (n = 0, 1, ...) completes phase n of
-            // kv_full[s]; slot 1's use 0 is K(0) alone, then pair j sits in slot j % 2 as
-            // that slot's use (j + (j & 1)) / 2.
-            int armed[kSlots] = {0, 0};
+            bool ok = p_ok;
             auto slot_use = [](int j) { return (j + (j & 1)) / 2; };
-            if (ok) ok = in_bounds(w.s0 + w.kv_lo >= 0 && w.s0 + w.kv_lo < p.L, p.status, abort_flag);
-            if (ok) {
-                mbar_arrive_expect_tx(&kv_full[1], Geo::kKVBytes);
-                ++armed[1];
-                for (int c = 0; c < Geo::kChunks; ++c)
-                    tma_load_3d(sK + 1 * Geo::kKVBytes + c * Geo::kChunkBytes, &p.tm_k, &kv_full[1], c * 64,
-                                w.s0 + w.kv_lo, zkv, pol_kv);
-            }
             for (int j = 0; j < n_kv && ok; ++j) {
                 const int sl = j & 1;
                 const int use = slot_use(j);
@@ -581,16 +599,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 const float g = p.gate[(size_t)w.b * p.L + w.s0 + pos];
                 gsig = 1.f / (1.f + expf(-g));
             }
-            #pragma unroll 1
+            // All of O_i's columns in one round trip to TMEM, then normalise and store.
+            uint32_t oall[D / 32][32];
+            __syncwarp();
+            #pragma unroll
+            for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, oall[c]);
+            #pragma unroll
+            for (int c = 0; c < D / 32; ++c) tmem_wait_ld(oall[c]);
+            #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
-                uint32_t orr[32];
-                __syncwarp();
-                tmem_ld32(tO + c * 32, orr);
-                tmem_wait_ld(orr);
-                if (!row_valid) continue;
+                if (!row_valid) break;
                 float vals[32];
                 #pragma unroll
-                for (int e = 0; e < 32; ++e) vals[e] = __uint_as_float(orr[e]) * inv_l;
+                for (int e = 0; e < 32; ++e) vals[e] = __uint_as_float(oall[c][e]) * inv_l;
                 int4* dst = reinterpret_cast<int4*>(orow + c * 32);
                 if (MODE == kModeGlobal && grow) {
                     int4* gdst = reinterpret_cast<int4*>(grow + c * 32);
