@@ -104,6 +104,27 @@ def algorithmic_bytes(d, Hq, Hkv, seqlens, counts, last_sel):
     return {"local": local, "global": glob}
 
 
+def executed_pairs(G, W, seqlens, cu_sel, sel, tile=128):
+    """(query, key) pairs per query head that the forward kernels' MMAs compute, masked ones
+    included: every CTA runs its two 128-row query tiles (two heads of one row tile when the
+    group size is even, else two consecutive row tiles or chunks of one head) against whole
+    128-key tiles from its first key to its last row's position."""
+    def ceil(a, b):
+        return -(-a // b)
+    per_cta = 1 if G % 2 == 0 else 2  # row tiles per head in one CTA
+    span = tile * per_cta
+    loc = glob = 0
+    for s, n in enumerate(seqlens):
+        for t0 in range(0, n, span):
+            last = min(n, t0 + span) - 1
+            loc += per_cta * tile * ceil(last + 1 - max(0, t0 - W + 1), tile) * tile
+        k = cu_sel[s + 1] - cu_sel[s]
+        for c0 in range(0, k, span):
+            last = sel[cu_sel[s] + min(k, c0 + span) - 1]
+            glob += per_cta * tile * ceil(last + 1, tile) * tile
+    return loc, glob
+
+
 def dense_causal_comparison(logo, q, k, v, w, ws, stream, dev, peak_burst, ms_step, reps=3):
     """The library's own dense causal attention on the same tensors: the local kernel with the
     window at least every sequence's length, so each query attends to its whole prefix.  Run
@@ -575,6 +596,8 @@ def main():
     sel_h = sel[:tot_sel].cpu().tolist()
     last_sel = [sel_h[cu_sel_h[s] + n - 1] if n > 0 else -1
                 for s, n in enumerate(cu_sel_h[i + 1] - cu_sel_h[i] for i in range(nseq))]
+    ex_loc, ex_glob = executed_pairs(w.Hq // w.Hkv, w.W, w.seqlens, cu_sel_h, sel_h)
+    ex_flop = {"local": 4 * w.d * Hq_r * ex_loc, "global": 4 * w.d * Hq_r * ex_glob}
     alg_bytes = algorithmic_bytes(w.d, Hq_r, k.shape[1], w.seqlens, [cu_sel_h[i + 1] - cu_sel_h[i] for i in range(nseq)],
                                   last_sel)
 
@@ -603,6 +626,9 @@ def main():
         per["global"].append(e[2].elapsed_time(e[3]))
     avg = {kk: sum(vv) / len(vv) for kk, vv in per.items()}
     ms_step = multirank.max_over_ranks(t_total_ms / args.steps, device=dev)  # slowest rank
+    step_ms = sorted(e[0].elapsed_time(e[3]) for e in evs)
+    step_median = multirank.max_over_ranks(statistics.median(step_ms), device=dev)
+    step_min = multirank.max_over_ranks(step_ms[0], device=dev)
     # head sharding: all ranks work on the same tokens; sequence sharding: on their own
     job_tokens = tokens if by_heads else int(multirank.sum_over_ranks(tokens, device=dev))
 
@@ -637,6 +663,8 @@ def main():
             "steps": args.steps,
             "warmup": args.warmup,
             "ms_per_step": ms_step,
+            "step_ms_median": step_median,
+            "step_ms_min": step_min,
             "higher_is_better": True,
             "scaling": "strong" if by_heads else "weak",
             "vs_baseline": None,
@@ -654,6 +682,10 @@ def main():
             "kernels_tflops": {"local": fl_local / (avg["local"] * 1e-3) / 1e12,
                                "global": fl_global / (avg["global"] * 1e-3) / 1e12},
             "useful_flop": {"local": fl_local, "global": fl_global},
+            "executed_flop": ex_flop,
+            "executed_tflops": {kk: ex_flop[kk] / (avg[kk] * 1e-3) / 1e12 for kk in ("local", "global")},
+            "useful_over_executed": {"local": fl_local / ex_flop["local"] if ex_flop["local"] else None,
+                                     "global": fl_global / ex_flop["global"] if ex_flop["global"] else None},
             "roofline": {"kernel": kern_name, "bound": "tensor", "achieved": achieved, "peak": peak_burst,
                          "unit": "TFLOP/s", "frac": achieved / peak_burst, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16 burst (sustained {peak_sust})",

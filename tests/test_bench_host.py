@@ -68,3 +68,29 @@ def test_cpu_baseline_reports_all_cores_and_one_thread():
     assert oracle.num_threads() == before  # restored after the single-thread sample
     if before > 1:
         assert r["single_thread"]["value"] > 0
+
+
+def _useful_local(L, W):
+    return sum(min(i + 1, W) for i in range(L))
+
+
+def test_executed_pairs_whole_tiles_and_union_for_odd_groups():
+    # even group: one 128-row tile per head and CTA; W >= L gives 1 + 2 key tiles for 256 rows
+    assert bench.executed_pairs(4, 256, [256], [0, 0], []) == (3 * 128 * 128, 0)
+    # odd group: two consecutive row tiles of one head share the union of their key ranges
+    loc, glob = bench.executed_pairs(3, 300, [700], [0, 3], [5, 400, 699])
+    assert loc == 2 * 128 * 128 * (2 + 4 + 4)
+    assert glob == 2 * 128 * 128 * 6  # one pair of chunks reaching position 699
+    # never below the useful pairs; equal when every tile is full and unmasked (W = 1 tile)
+    for G, W, n in [(2, 4096, 32768), (1, 300, 1000), (4, 1, 129), (5, 17, 300)]:
+        loc, _ = bench.executed_pairs(G, W, [n], [0, 0], [])
+        assert loc >= _useful_local(n, W)
+    loc, _ = bench.executed_pairs(2, 10 ** 6, [512], [0, 0], [])
+    assert loc == 128 * 128 * (1 + 2 + 3 + 4)
+
+
+def test_executed_pairs_packed_sequences_are_independent():
+    a = bench.executed_pairs(4, 64, [300], [0, 2], [10, 299])
+    b = bench.executed_pairs(4, 64, [1000], [0, 1], [512])
+    both = bench.executed_pairs(4, 64, [300, 1000], [0, 2, 3], [10, 299, 512])
+    assert both == (a[0] + b[0], a[1] + b[1])
