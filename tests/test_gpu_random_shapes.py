@@ -39,7 +39,7 @@ def draw_case(seed):
     return B, Hkv * G, Hkv, L, d, W, ratio, seqlens
 
 
-CASES = list(range(12))
+CASES = list(range(24))
 
 
 @pytest.mark.parametrize("seed", CASES)
@@ -61,7 +61,7 @@ def test_forward_random_shape(seed):
           max_abs=MAX_ABS * max(1.0, r.abs().max().item() / 4.0))
 
 
-@pytest.mark.parametrize("seed", CASES[:6])
+@pytest.mark.parametrize("seed", CASES[:12])
 def test_backward_random_shape(seed):
     from tests.test_gpu_backward import close as close_grad, gpu_run
 
