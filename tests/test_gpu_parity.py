@@ -280,6 +280,19 @@ def test_select_random_ties_specials(seed):
         assert _select_gpu(g, ratio) == oracle.select(g, ratio).tolist()
 
 
+def test_select_long_sequence_streams_keys():
+    """A sequence whose slices exceed what the selection keeps in shared memory: every pass
+    re-reads the logits (heavy ties and the special values as above)."""
+    n = 8 * 40960 + 12345
+    gen = torch.Generator().manual_seed(11)
+    g = (torch.randn(n, generator=gen) * 4).round() / 4
+    specials = torch.tensor([0.0, -0.0, float("inf"), float("-inf"), float("nan")])
+    idx = torch.randint(0, n, (n // 50,), generator=gen)
+    g[idx] = specials[torch.randint(0, len(specials), (idx.numel(),), generator=gen)]
+    for ratio in (0.05, 0.2, 0.5):
+        assert _select_gpu(g, ratio) == oracle.select(g, ratio).tolist()
+
+
 # --------------------------------------------------------------------------
 # the named workloads at full size, in the benchmark's launch configuration
 # --------------------------------------------------------------------------

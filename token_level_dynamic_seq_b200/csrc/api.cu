@@ -405,7 +405,8 @@ logo_status logo_select(const float* gate, const logo_shape* shape, double ratio
         e = cudaMemsetAsync(cu_sel, 0, sizeof(int32_t) * (size_t)(g.nseq + 1), static_cast<cudaStream_t>(stream));
     } else {
         NvtxRange range("logo select");
-        e = logo::launch_select(gate, g.cu, g.nseq, g.L, ratio, sel_idx, cu_sel, static_cast<cudaStream_t>(stream));
+        e = logo::launch_select(gate, g.cu, g.nseq, g.L, g.max_len, ratio, sel_idx, cu_sel,
+                                static_cast<cudaStream_t>(stream));
     }
     return e == cudaSuccess ? LOGO_OK : cuda_fail(e, "select launch");
 }

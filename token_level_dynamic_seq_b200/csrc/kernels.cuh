@@ -82,8 +82,8 @@ struct alignas(64) AttnParams {
     int sel_stride;
 };
 
-cudaError_t launch_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, double ratio,
-                          int32_t* sel_idx, int32_t* cu_sel, cudaStream_t stream);
+cudaError_t launch_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, int max_len,
+                          double ratio, int32_t* sel_idx, int32_t* cu_sel, cudaStream_t stream);
 
 cudaError_t launch_threshold_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, const float* tau,
                                     int max_selected, int32_t* counts, int32_t* sel_idx, int32_t* cu_sel,

@@ -8,21 +8,25 @@
 // Architecture of Conditional Attention" (a yes/no routing decision for each
 // position, about one in five going global).
 //
-// One 1024-thread CTA per sequence:
+// Each sequence is spread over a cluster of kClusterCtas CTAs, CTA r holding the r-th
+// contiguous slice of the sequence:
 //  1. map each fp32 logit to a 32-bit key whose unsigned order is the
-//     selection order (-0 folded onto +0, every NaN to 0, below -inf); when
-//     the sequence fits (kResidentKeys keys) the keys stay in shared memory
-//     for every later pass, otherwise each pass re-reads the logits;
-//  2. radix-select the k-th largest key T with four 8-bit passes; each warp
-//     counts into its own shared-memory histogram (no contention between
-//     warps; the lanes still matching the prefix merge equal digits with
-//     __match_any_sync, warps with no such lane skip it), and
-//     the 32 histograms are summed before the digit is chosen; this also
-//     yields how many keys equal to T must be taken;
-//  3. stream-compact in ascending position order, 4096 elements per step:
-//     a block-wide scan places the selected positions; when only some of the
-//     keys equal to T are taken, a second scan ranks those keys first (the
-//     lowest positions win).
+//     selection order (-0 folded onto +0, every NaN to 0, below -inf); a slice
+//     of up to kSliceResident keys stays in shared memory for every later pass,
+//     a longer one is re-read from the logits each pass;
+//  2. radix-select the k-th largest key T with four 8-bit passes: each CTA
+//     counts its slice into a shared-memory histogram, and after a cluster
+//     barrier every CTA sums the cluster's histograms through distributed
+//     shared memory and takes the same digit; the last pass also gives how
+//     many keys equal to T there are, and how many of them must be taken;
+//  3. stream-compact in ascending position order: each CTA's keys above T and
+//     equal to T are counted and exchanged the same way, so a slice's selected
+//     positions go after those of the lower-ranked slices, and the keys equal to
+//     T are taken lowest position first up to the count.
+// The controller step of the threshold form (further down) finds one order
+// statistic of a whole batch with the same passes inside one 1024-thread CTA
+// (radix_kth_largest: per-warp histograms, lanes with equal digits merged with
+// __match_any_sync).
 // Integer work only, so the result is bit-exact.
 #include <cuda_runtime.h>
 
@@ -37,8 +41,6 @@ namespace {
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kItems = 4;
-constexpr int kResidentKeys = 40960;  // 160 KB of keys kept in shared memory
-constexpr size_t kSelDynSmem = (size_t)kResidentKeys * 4 + (size_t)kSelWarps * 256 * 4;
 
 __device__ __forceinline__ uint32_t gate_key(float f)
 {
@@ -167,19 +169,98 @@ __device__ KthResult radix_kth_largest(KeyAt key_at, long long len, long long k,
     return r;
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const float* __restrict__ gate,
-                                                                  const int32_t* __restrict__ cu_seqlens,
-                                                                  int nseq, int L, double ratio,
-                                                                  int32_t* __restrict__ sel_idx,
-                                                                  int32_t* __restrict__ cu_sel)
-{
-    extern __shared__ uint32_t dyn_smem[];
-    uint32_t* keys_s = dyn_smem;                            // kResidentKeys
-    uint32_t* whist = dyn_smem + kResidentKeys;             // [kSelWarps][256]
-    __shared__ uint32_t hist[256];
-    __shared__ int warp_buf[32];
+// ---------------------------------------------------------------- cluster form
+//
+// The top-k selection: each sequence spread over a cluster of kClusterCtas CTAs, CTA r of the
+// cluster holding the r-th contiguous slice of the sequence's keys.  Every radix pass counts
+// the slice into a CTA histogram, one cluster barrier later each CTA sums all the cluster's
+// histograms through distributed shared memory and takes the same digit; the compaction places
+// each CTA's slice after the selected keys of the lower-ranked slices (their counts are read the
+// same way), so positions still come out ascending and ties still go to the lower position.
+// Every CTA of a cluster works on the same sequence and takes the same branches, so all of them
+// reach every cluster barrier.
 
-    const int s = blockIdx.x;
+constexpr int kClusterCtas = 8;
+constexpr int kCThreads = 512;
+constexpr int kCWarps = kCThreads / 32;
+constexpr int kSliceResident = 40960;  // keys of one slice kept in shared memory (160 KB)
+
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address of the same shared-memory variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_map(const void* local, uint32_t rank)
+{
+    uint32_t a = (uint32_t)__cvta_generic_to_shared(local), r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ long long ld_cluster_s64(uint32_t addr)
+{
+    long long v;
+    asm volatile("ld.shared::cluster.s64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// Exclusive prefix sum over a kCThreads block; `total` receives the block sum.
+__device__ __forceinline__ int cblock_exclusive_scan(int v, int* warp_buf, int& total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+    #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_buf[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int s = lane < kCWarps ? warp_buf[lane] : 0;
+        #pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += y;
+        }
+        if (lane < kCWarps) warp_buf[lane] = s;  // inclusive
+    }
+    __syncthreads();
+    const int before = warp ? warp_buf[warp - 1] : 0;
+    total = warp_buf[kCWarps - 1];
+    __syncthreads();  // warp_buf may be reused right after
+    return before + x - v;
+}
+
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kCThreads)
+    select_cluster_kernel(const float* __restrict__ gate, const int32_t* __restrict__ cu_seqlens, int nseq, int L,
+                          double ratio, int32_t* __restrict__ sel_idx, int32_t* __restrict__ cu_sel, int resident_cap)
+{
+    extern __shared__ uint32_t slice_keys[];  // resident_cap keys (at most kSliceResident)
+    __shared__ uint32_t hist[2][256];         // this slice's counts, alternating between passes
+    __shared__ uint32_t tot[256];             // the cluster's counts
+    __shared__ long long cnt[2];              // keys of this slice above T, equal to T
+    __shared__ int warp_buf[32];
+    __shared__ uint32_t sh_digit, sh_bin_count;
+    __shared__ long long sh_remaining, sh_sel_before, sh_eq_quota;
+
+    const uint32_t rank = cluster_ctarank();
+    const int s = blockIdx.y;
     const int tid = threadIdx.x;
     long long start, len, out_off;
     if (cu_seqlens) {
@@ -192,66 +273,150 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const float* _
         len = L;
         out_off = (long long)s * budget_count(ratio, L);
     }
-    const long long k = budget_count(ratio, len);
-    if (tid == 0) {
+    const long long k = budget_count(ratio, len);  // the same in every CTA of the cluster
+    if (rank == 0 && tid == 0) {
         cu_sel[s + 1] = (int32_t)(out_off + k);
         if (s == 0) cu_sel[0] = 0;
     }
     if (k <= 0) return;
-    const float* g = gate + start;
+    const long long lo = len * rank / kClusterCtas, hi = len * (rank + 1) / kClusterCtas, n = hi - lo;
+    const float* g = gate + start + lo;
     int32_t* out = sel_idx + out_off;
     if (k == len) {
-        for (long long i = tid; i < len; i += kSelThreads) out[i] = (int32_t)i;
+        for (long long i = tid; i < n; i += kCThreads) out[lo + i] = (int32_t)(lo + i);
         return;
     }
-    const bool resident = len <= kResidentKeys;
-    if (resident) {
-        for (long long i = tid; i < len; i += kSelThreads) keys_s[i] = gate_key(__ldg(g + i));
+    const bool resident = n <= resident_cap;  // the launch sized the array for the longest sequence
+    if (resident)
+        for (long long i = tid; i < n; i += kCThreads) slice_keys[i] = gate_key(__ldg(g + i));
+    auto key_at = [&](long long i) -> uint32_t { return resident ? slice_keys[i] : gate_key(__ldg(g + i)); };
+
+    // ---- radix select of the k-th largest key over the whole sequence
+    uint32_t prefix = 0, mask = 0;
+    long long remaining = k;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass, b = pass & 1;
+        if (tid < 256) hist[b][tid] = 0;
         __syncthreads();
+        for (long long i = tid; i < n; i += kCThreads) {
+            const uint32_t key = key_at(i);
+            if ((key & mask) == prefix) atomicAdd(&hist[b][(key >> shift) & 255u], 1u);
+        }
+        // Every slice's counts of this pass are complete.  A CTA writes hist[b] again two
+        // passes later, after the next barrier, which no CTA passes before it has read these.
+        cluster_sync_all();
+        if (tid < 256) {
+            uint32_t c = 0;
+            #pragma unroll
+            for (int r = 0; r < kClusterCtas; ++r) c += ld_cluster_u32(cluster_map(&hist[b][tid], (uint32_t)r));
+            tot[tid] = c;
+        }
+        __syncthreads();
+        if (tid < 32) {
+            // lane l owns bins 255-8l .. 248-8l (descending)
+            const int lane = tid;
+            uint32_t c[8];
+            uint32_t sum = 0;
+            #pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                c[t] = tot[255 - 8 * lane - t];
+                sum += c[t];
+            }
+            uint32_t incl = sum;
+            #pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const long long excl = (long long)(incl - sum);
+            if (excl < remaining && remaining <= excl + (long long)sum) {
+                long long acc = excl;
+                #pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    if (acc + (long long)c[t] >= remaining) {
+                        sh_digit = 255u - 8u * lane - t;
+                        sh_remaining = remaining - acc;
+                        sh_bin_count = c[t];
+                        break;
+                    }
+                    acc += c[t];
+                }
+            }
+        }
+        __syncthreads();
+        prefix |= sh_digit << shift;
+        mask |= 255u << shift;
+        remaining = sh_remaining;
     }
-    auto key_at = [&](long long i) -> uint32_t { return resident ? keys_s[i] : gate_key(__ldg(g + i)); };
+    const uint32_t T = prefix;                    // the k-th largest key
+    const long long take_eq = remaining;          // how many keys equal to T are selected
+    const bool all_eq = take_eq == (long long)sh_bin_count;
 
-    // ---- radix select of the k-th largest key
-    const KthResult kr = radix_kth_largest(key_at, len, k, whist, hist);
-    const uint32_t T = kr.key;              // the k-th largest key
-    const long long take_eq = kr.take_eq;   // how many keys equal to T are selected
-    // Usually every key equal to T is taken; then "key >= T" decides alone and one
-    // scan per chunk suffices.
-    const bool all_eq = take_eq == kr.eq_count;
+    // ---- this slice's keys above and equal to T, then its place among the cluster's slices
+    int n_gt = 0, n_eq = 0;
+    for (long long i = tid; i < n; i += kCThreads) {
+        const uint32_t key = key_at(i);
+        n_gt += key > T ? 1 : 0;
+        n_eq += key == T ? 1 : 0;
+    }
+    int tot_gt, tot_eq;
+    cblock_exclusive_scan(n_gt, warp_buf, tot_gt);
+    cblock_exclusive_scan(n_eq, warp_buf, tot_eq);
+    if (tid == 0) {
+        cnt[0] = tot_gt;
+        cnt[1] = tot_eq;
+    }
+    cluster_sync_all();
+    if (tid == 0) {
+        long long gt_before = 0, eq_before = 0;
+        for (uint32_t r = 0; r < rank; ++r) {
+            gt_before += ld_cluster_s64(cluster_map(&cnt[0], r));
+            eq_before += ld_cluster_s64(cluster_map(&cnt[1], r));
+        }
+        const long long eq_taken_before = all_eq ? eq_before : (eq_before < take_eq ? eq_before : take_eq);
+        sh_sel_before = gt_before + eq_taken_before;
+        const long long q = all_eq ? (long long)tot_eq : take_eq - eq_taken_before;
+        sh_eq_quota = q < 0 ? 0 : (q > tot_eq ? tot_eq : q);
+    }
+    __syncthreads();
+    const long long eq_quota = sh_eq_quota;
+    const bool take_all_eq = eq_quota == (long long)tot_eq;
 
-    // ---- compaction in ascending position order
-    long long eq_seen = 0, written = 0;
-    for (long long chunk = 0; chunk < len; chunk += (long long)kSelThreads * kItems) {
+    // ---- compaction of the slice in ascending position order
+    long long eq_seen = 0, written = sh_sel_before;
+    for (long long chunk = 0; chunk < n; chunk += (long long)kCThreads * kItems) {
         const long long i0 = chunk + (long long)tid * kItems;
         uint32_t keys[kItems];
-        int n_eq = 0;
+        int n_eq_t = 0;
         #pragma unroll
         for (int t = 0; t < kItems; ++t) {
-            keys[t] = (i0 + t < len) ? key_at(i0 + t) : 0u;
-            n_eq += (i0 + t < len && keys[t] == T) ? 1 : 0;
+            keys[t] = (i0 + t < n) ? key_at(i0 + t) : 0u;
+            n_eq_t += (i0 + t < n && keys[t] == T) ? 1 : 0;
         }
         int eq_total = 0, eq_before = 0;
-        if (!all_eq) eq_before = block_exclusive_scan(n_eq, warp_buf, eq_total);
+        if (!take_all_eq) eq_before = cblock_exclusive_scan(n_eq_t, warp_buf, eq_total);
         bool sel[kItems];
         int n_sel = 0, eq_run = 0;
         #pragma unroll
         for (int t = 0; t < kItems; ++t) {
-            const bool in = i0 + t < len;
+            const bool in = i0 + t < n;
             const bool gt = in && keys[t] > T;
             const bool eq = in && keys[t] == T;
-            sel[t] = gt || (eq && (all_eq || (eq_seen + eq_before + eq_run) < take_eq));
+            sel[t] = gt || (eq && (take_all_eq || (eq_seen + eq_before + eq_run) < eq_quota));
             eq_run += eq ? 1 : 0;
             n_sel += sel[t] ? 1 : 0;
         }
         int sel_total;
-        const int sel_before = block_exclusive_scan(n_sel, warp_buf, sel_total);
+        const int sel_before = cblock_exclusive_scan(n_sel, warp_buf, sel_total);
         int o = 0;
         #pragma unroll
         for (int t = 0; t < kItems; ++t)
-            if (sel[t]) out[written + sel_before + (o++)] = (int32_t)(i0 + t);
+            if (sel[t]) out[written + sel_before + (o++)] = (int32_t)(lo + i0 + t);
         eq_seen += eq_total;
         written += sel_total;
     }
+    // No CTA leaves while another may still read its shared memory.
+    cluster_sync_all();
 }
 
 // ---------------------------------------------------------------- threshold form
@@ -405,15 +570,19 @@ cudaError_t launch_threshold_update(const float* gate, const int32_t* cu_seqlens
     return cudaGetLastError();
 }
 
-cudaError_t launch_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, double ratio,
-                          int32_t* sel_idx, int32_t* cu_sel, cudaStream_t stream)
+cudaError_t launch_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, int max_len,
+                          double ratio, int32_t* sel_idx, int32_t* cu_sel, cudaStream_t stream)
 {
     if (nseq <= 0) return cudaSuccess;
-    cudaError_t e =
-        cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelDynSmem);
+    // One cluster of kClusterCtas CTAs per sequence; its slices of at most kSliceResident keys
+    // stay in shared memory.
+    const long long slice = ((long long)(max_len > 0 ? max_len : 1) + kClusterCtas - 1) / kClusterCtas;
+    const int cap = (int)(slice < kSliceResident ? slice : kSliceResident);
+    const size_t smem = (size_t)cap * 4;
+    cudaError_t e = cudaFuncSetAttribute(select_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    select_topk_kernel<<<nseq, kSelThreads, kSelDynSmem, stream>>>(gate, cu_seqlens, nseq, L, ratio, sel_idx,
-                                                                   cu_sel);
+    select_cluster_kernel<<<dim3(kClusterCtas, nseq), kCThreads, smem, stream>>>(gate, cu_seqlens, nseq, L, ratio,
+                                                                                 sel_idx, cu_sel, cap);
     return cudaGetLastError();
 }
 
