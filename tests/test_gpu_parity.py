@@ -6,6 +6,7 @@ compare every element (several 128-row tiles and a ragged tail); the
 full-size workloads, run in the benchmark's launch configuration, compare the
 selection in full and a sample of rows the oracle computes one by one.
 """
+import itertools
 import math
 import random
 
@@ -278,6 +279,27 @@ def test_select_random_ties_specials(seed):
     g[idx] = specials[torch.randint(0, len(specials), (idx.numel(),), generator=gen)]
     for ratio in (0.0, 0.05, 0.2, 0.5, 0.999, 1.0):
         assert _select_gpu(g, ratio) == oracle.select(g, ratio).tolist()
+
+
+def test_select_many_short_packed_sequences():
+    """A packed batch of 257 short sequences (0 to 300 tokens, ties and special values): one
+    cluster per sequence, each of a single CTA at these lengths; the list and cu_sel bit for bit."""
+    rng = random.Random(3)
+    lens = [rng.choice([0, 1, 2, 7, 8, 9, rng.randrange(3, 300)]) for _ in range(257)]
+    T = sum(lens)
+    gen = torch.Generator().manual_seed(3)
+    g = (torch.randn(T, generator=gen) * 2).round() / 2
+    g[torch.randint(0, T, (T // 40,), generator=gen)] = float("nan")
+    cu = torch.tensor([0] + list(itertools.accumulate(lens)), dtype=torch.int32)
+    ratio = 0.3
+    cu_dev = cu.cuda()
+    sh = logo.Shape(1, 1, 1, T, 128, cu_dev.data_ptr(), len(lens), max(lens))
+    ws = logo.workspace(sh, ratio, torch.device("cuda"))
+    sel, cu_sel = logo.select(g.view(1, T).cuda(), sh, ratio, ws)
+    logo.check(ws)
+    got = sel_lists(sel, cu_sel)
+    want = [oracle.select(g[int(cu[s]):int(cu[s + 1])], ratio).tolist() for s in range(len(lens))]
+    assert got == want
 
 
 def test_select_long_sequence_streams_keys():

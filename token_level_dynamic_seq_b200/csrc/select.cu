@@ -8,8 +8,9 @@
 // Architecture of Conditional Attention" (a yes/no routing decision for each
 // position, about one in five going global).
 //
-// Each sequence is spread over a cluster of kClusterCtas CTAs, CTA r holding the r-th
-// contiguous slice of the sequence:
+// Each sequence is spread over a cluster of up to kClusterCtas CTAs (one CTA per 4096 tokens
+// of the longest sequence, rounded up to a power of two), CTA r holding the r-th contiguous
+// slice of the sequence:
 //  1. map each fp32 logit to a 32-bit key whose unsigned order is the
 //     selection order (-0 folded onto +0, every NaN to 0, below -inf); a slice
 //     of up to kSliceResident keys stays in shared memory for every later pass,
@@ -171,8 +172,8 @@ __device__ KthResult radix_kth_largest(KeyAt key_at, long long len, long long k,
 
 // ---------------------------------------------------------------- cluster form
 //
-// The top-k selection: each sequence spread over a cluster of kClusterCtas CTAs, CTA r of the
-// cluster holding the r-th contiguous slice of the sequence's keys.  Every radix pass counts
+// The top-k selection: each sequence spread over a cluster of up to kClusterCtas CTAs, CTA r of
+// the cluster holding the r-th contiguous slice of the sequence's keys.  Every radix pass counts
 // the slice into a CTA histogram, one cluster barrier later each CTA sums all the cluster's
 // histograms through distributed shared memory and takes the same digit; the compaction places
 // each CTA's slice after the selected keys of the lower-ranked slices (their counts are read the
@@ -180,7 +181,8 @@ __device__ KthResult radix_kth_largest(KeyAt key_at, long long len, long long k,
 // Every CTA of a cluster works on the same sequence and takes the same branches, so all of them
 // reach every cluster barrier.
 
-constexpr int kClusterCtas = 8;
+constexpr int kClusterCtas = 8;        // largest cluster
+constexpr int kKeysPerCta = 4096;      // a cluster gets one CTA per this many keys (power of two)
 constexpr int kCThreads = 512;
 constexpr int kCWarps = kCThreads / 32;
 constexpr int kSliceResident = 40960;  // keys of one slice kept in shared memory (160 KB)
@@ -188,6 +190,13 @@ constexpr int kSliceResident = 40960;  // keys of one slice kept in shared memor
 __device__ __forceinline__ void cluster_sync_all()
 {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_nctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
 }
 
 __device__ __forceinline__ uint32_t cluster_ctarank()
@@ -247,7 +256,7 @@ __device__ __forceinline__ int cblock_exclusive_scan(int v, int* warp_buf, int& 
     return before + x - v;
 }
 
-__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kCThreads)
+__global__ void __launch_bounds__(kCThreads)
     select_cluster_kernel(const float* __restrict__ gate, const int32_t* __restrict__ cu_seqlens, int nseq, int L,
                           double ratio, int32_t* __restrict__ sel_idx, int32_t* __restrict__ cu_sel, int resident_cap)
 {
@@ -260,6 +269,7 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kCThreads
     __shared__ long long sh_remaining, sh_sel_before, sh_eq_quota;
 
     const uint32_t rank = cluster_ctarank();
+    const uint32_t nranks = cluster_nctarank();  // the launch's cluster size, 1 to kClusterCtas
     const int s = blockIdx.y;
     const int tid = threadIdx.x;
     long long start, len, out_off;
@@ -279,7 +289,7 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kCThreads
         if (s == 0) cu_sel[0] = 0;
     }
     if (k <= 0) return;
-    const long long lo = len * rank / kClusterCtas, hi = len * (rank + 1) / kClusterCtas, n = hi - lo;
+    const long long lo = len * rank / nranks, hi = len * (rank + 1) / nranks, n = hi - lo;
     const float* g = gate + start + lo;
     int32_t* out = sel_idx + out_off;
     if (k == len) {
@@ -307,8 +317,7 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kCThreads
         cluster_sync_all();
         if (tid < 256) {
             uint32_t c = 0;
-            #pragma unroll
-            for (int r = 0; r < kClusterCtas; ++r) c += ld_cluster_u32(cluster_map(&hist[b][tid], (uint32_t)r));
+            for (uint32_t r = 0; r < nranks; ++r) c += ld_cluster_u32(cluster_map(&hist[b][tid], r));
             tot[tid] = c;
         }
         __syncthreads();
@@ -574,16 +583,30 @@ cudaError_t launch_select(const float* gate, const int32_t* cu_seqlens, int nseq
                           double ratio, int32_t* sel_idx, int32_t* cu_sel, cudaStream_t stream)
 {
     if (nseq <= 0) return cudaSuccess;
-    // One cluster of kClusterCtas CTAs per sequence; its slices of at most kSliceResident keys
-    // stay in shared memory.
-    const long long slice = ((long long)(max_len > 0 ? max_len : 1) + kClusterCtas - 1) / kClusterCtas;
+    // One cluster per sequence, of one CTA per kKeysPerCta keys of the longest sequence (a power
+    // of two, at most kClusterCtas); its slices of at most kSliceResident keys stay in shared
+    // memory.
+    const long long ml = max_len > 0 ? max_len : 1;
+    int ctas = 1;
+    while (ctas < kClusterCtas && (long long)ctas * kKeysPerCta < ml) ctas *= 2;
+    const long long slice = (ml + ctas - 1) / ctas;
     const int cap = (int)(slice < kSliceResident ? slice : kSliceResident);
     const size_t smem = (size_t)cap * 4;
     cudaError_t e = cudaFuncSetAttribute(select_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    select_cluster_kernel<<<dim3(kClusterCtas, nseq), kCThreads, smem, stream>>>(gate, cu_seqlens, nseq, L, ratio,
-                                                                                 sel_idx, cu_sel, cap);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ctas, nseq);
+    cfg.blockDim = dim3(kCThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = ctas;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, select_cluster_kernel, gate, cu_seqlens, nseq, L, ratio, sel_idx, cu_sel, cap);
 }
 
 }  // namespace logo
