@@ -159,6 +159,43 @@ def dense_causal_comparison(logo, q, k, v, w, ws, stream, dev, peak_burst, ms_st
         return {"error": str(e)[:300]}
 
 
+def threshold_form_timing(logo, g, shape, w, ws, stream, dev, reps=20):
+    """The threshold form of the budget rule on the same gate: one controller step (the batch
+    target, beta = 1, so the threshold lands on it) and the selection of every position above the
+    threshold, each timed alone with CUDA events; a failure is reported in the line."""
+    try:
+        import torch
+        nseq = len(w.seqlens)
+        cap = max(w.seqlens)  # a sequence may hold more than its share of the batch's top logits
+        tau = torch.zeros(1, dtype=torch.float32, device=dev)
+        sel = torch.empty(max(1, nseq * cap), dtype=torch.int32, device=dev)
+        cu_sel = torch.empty(nseq + 1, dtype=torch.int32, device=dev)
+        target = torch.empty(1, dtype=torch.float32, device=dev)
+
+        def update():
+            logo.threshold_update(g, shape, w.ratio, 1.0, tau, ws, target=target, stream=stream)
+
+        def select():
+            logo.select_threshold(g, shape, tau, cap, ws, sel, cu_sel, stream=stream)
+
+        out = {}
+        for name, fn in (("update_ms", update), ("select_ms", select)):
+            for _ in range(3):
+                fn()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            ev[0].record(stream)
+            for _ in range(reps):
+                fn()
+            ev[1].record(stream)
+            torch.cuda.synchronize(dev)
+            out[name] = ev[0].elapsed_time(ev[1]) / reps
+        logo.check(ws, stream)
+        out["selected"] = int(cu_sel[-1].item())
+        return out
+    except Exception as e:  # reported, never fatal for the bench line
+        return {"error": str(e)[:300]}
+
+
 def traffic_record():
     """DRAM bytes per launch from the committed ncu summary, if taken on the current kernel source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -652,6 +689,7 @@ def main():
     if rank == 0:
         dense = None if args.profile else dense_causal_comparison(logo, q, k, v, w, ws, stream, dev, peak_burst,
                                                                    ms_step)
+        thr = None if args.profile else threshold_form_timing(logo, g, shape, w, ws, stream, dev)
         cpu = None
         if world == 1 and not (args.no_cpu_baseline or args.profile):
             cpu = cpu_baseline(w)
@@ -702,6 +740,7 @@ def main():
             "wall_s_timed": t_wall,
             "cpu_baseline": cpu,
             "comparisons": {"dense_causal": dense},
+            "threshold_form": thr,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

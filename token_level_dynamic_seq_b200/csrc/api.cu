@@ -659,8 +659,8 @@ logo_status logo_select_threshold(const float* gate, const logo_shape* shape, co
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int32_t* counts = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kWsHeaderBytes);
     NvtxRange range("logo threshold select");
-    cudaError_t e = logo::launch_threshold_select(gate, g.cu, g.nseq, g.L, tau, max_selected, counts, sel_idx, cu_sel,
-                                                  static_cast<uint32_t*>(ws), s);
+    cudaError_t e = logo::launch_threshold_select(gate, g.cu, g.nseq, g.L, g.max_len, tau, max_selected, counts,
+                                                  sel_idx, cu_sel, static_cast<uint32_t*>(ws), s);
     return e == cudaSuccess ? LOGO_OK : cuda_fail(e, "threshold select launch");
 }
 
@@ -679,7 +679,8 @@ logo_status logo_threshold_update(const float* gate, const logo_shape* shape, do
     if (g.L > 0 && (st = check_ptr(gate, "gate")) != LOGO_OK) return st;
     const long long n_fixed = (long long)g.B * g.L;
     NvtxRange range("logo threshold update");
-    cudaError_t e = logo::launch_threshold_update(gate, g.cu, g.nseq, n_fixed, ratio, beta, tau, target,
+    const long long n_all = g.cu ? (long long)g.L : n_fixed;  // packed: L is the total token count
+    cudaError_t e = logo::launch_threshold_update(gate, g.cu, g.nseq, n_all, n_fixed, ratio, beta, tau, target,
                                                   static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? LOGO_OK : cuda_fail(e, "threshold update launch");
 }

@@ -85,12 +85,13 @@ struct alignas(64) AttnParams {
 cudaError_t launch_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, int max_len,
                           double ratio, int32_t* sel_idx, int32_t* cu_sel, cudaStream_t stream);
 
-cudaError_t launch_threshold_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, const float* tau,
-                                    int max_selected, int32_t* counts, int32_t* sel_idx, int32_t* cu_sel,
-                                    uint32_t* status, cudaStream_t stream);
+cudaError_t launch_threshold_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, int max_len,
+                                    const float* tau, int max_selected, int32_t* counts, int32_t* sel_idx,
+                                    int32_t* cu_sel, uint32_t* status, cudaStream_t stream);
 
-cudaError_t launch_threshold_update(const float* gate, const int32_t* cu_seqlens, int nseq, long long n_fixed,
-                                    double ratio, float beta, float* tau, float* target_out, cudaStream_t stream);
+cudaError_t launch_threshold_update(const float* gate, const int32_t* cu_seqlens, int nseq, long long n_all,
+                                    long long n_fixed, double ratio, float beta, float* tau, float* target_out,
+                                    cudaStream_t stream);
 
 // Decode step (decode.cu).
 constexpr int kDecChunk = 512;  // cache positions per partial state

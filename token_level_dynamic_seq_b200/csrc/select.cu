@@ -24,14 +24,14 @@
 //     equal to T are counted and exchanged the same way, so a slice's selected
 //     positions go after those of the lower-ranked slices, and the keys equal to
 //     T are taken lowest position first up to the count.
-// The controller step of the threshold form (further down) finds one order
-// statistic of a whole batch with the same passes inside one 1024-thread CTA
-// (radix_kth_largest: per-warp histograms, lanes with equal digits merged with
-// __match_any_sync).
+// The threshold form (further down) counts and compacts the positions above a
+// threshold on the same clusters, and its controller step finds one order
+// statistic of the whole batch with the same radix passes.
 // Integer work only, so the result is bit-exact.
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <utility>
 
 #include "kernels.cuh"
 
@@ -39,8 +39,6 @@ namespace logo {
 
 namespace {
 
-constexpr int kSelThreads = 1024;
-constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kItems = 4;
 
 __device__ __forceinline__ uint32_t gate_key(float f)
@@ -49,125 +47,6 @@ __device__ __forceinline__ uint32_t gate_key(float f)
     if ((b & 0x7FFFFFFFu) > 0x7F800000u) return 0u;  // NaN ranks below everything
     if (b == 0x80000000u) b = 0u;                      // -0 equals +0
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-
-// Exclusive prefix sum over the block; `total` receives the block sum.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_buf, int& total)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = v;
-    #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) warp_buf[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        int s = warp_buf[lane];
-        #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, s, o);
-            if (lane >= o) s += y;
-        }
-        warp_buf[lane] = s;  // inclusive
-    }
-    __syncthreads();
-    const int before = warp ? warp_buf[warp - 1] : 0;
-    total = warp_buf[kSelWarps - 1];
-    __syncthreads();  // warp_buf may be reused right after
-    return before + x - v;
-}
-
-struct KthResult {
-    uint32_t key;        // the k-th largest key
-    long long take_eq;   // how many keys equal to it are among the k largest
-    long long eq_count;  // how many keys equal to it there are
-};
-
-// Radix select over `len` keys (key_at(i)) with four 8-bit passes, 1 <= k <= len.
-// Called by all threads of a 1024-thread block; whist holds [kSelWarps][256]
-// per-warp histograms, hist 256 words.  Each warp counts into its own histogram
-// (the lanes still matching the prefix merge equal digits with __match_any_sync,
-// warps with no such lane skip it); the 32 histograms are summed before the
-// digit is chosen.
-template <typename KeyAt>
-__device__ KthResult radix_kth_largest(KeyAt key_at, long long len, long long k, uint32_t* whist, uint32_t* hist)
-{
-    __shared__ uint32_t sh_digit;
-    __shared__ long long sh_remaining;
-    __shared__ uint32_t sh_bin_count;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint32_t prefix = 0, mask = 0;
-    long long remaining = k;
-    uint32_t* myhist = whist + warp * 256;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = lane; i < 256; i += 32) myhist[i] = 0;
-        __syncwarp();
-        for (long long base = (long long)warp * 32; base < len; base += kSelThreads) {
-            const long long i = base + lane;
-            const bool in = i < len;
-            const uint32_t key = in ? key_at(i) : 0u;
-            const bool match = in && ((key & mask) == prefix);
-            const uint32_t digit = (key >> shift) & 255u;
-            const uint32_t active = __ballot_sync(0xffffffffu, match);
-            if (match) {
-                const uint32_t peers = __match_any_sync(active, digit);
-                // one lane per distinct digit, and only this warp writes this histogram
-                if (lane == __ffs(peers) - 1) myhist[digit] += (uint32_t)__popc(peers);
-            }
-            __syncwarp();
-        }
-        __syncthreads();
-        if (tid < 256) {
-            uint32_t c = 0;
-            #pragma unroll 8
-            for (int w = 0; w < kSelWarps; ++w) c += whist[w * 256 + tid];
-            hist[tid] = c;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            // lane l owns bins 255-8l .. 248-8l (descending); after the last pass the
-            // chosen bin's count is the number of keys equal to the result
-            uint32_t c[8];
-            uint32_t sum = 0;
-            #pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                c[t] = hist[255 - 8 * lane - t];
-                sum += c[t];
-            }
-            uint32_t incl = sum;
-            #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            const long long excl = (long long)(incl - sum);
-            if (excl < remaining && remaining <= excl + (long long)sum) {
-                long long acc = excl;
-                #pragma unroll
-                for (int t = 0; t < 8; ++t) {
-                    if (acc + (long long)c[t] >= remaining) {
-                        sh_digit = 255u - 8u * lane - t;
-                        sh_remaining = remaining - acc;
-                        sh_bin_count = c[t];
-                        break;
-                    }
-                    acc += c[t];
-                }
-            }
-        }
-        __syncthreads();
-        prefix |= sh_digit << shift;
-        mask |= 255u << shift;
-        remaining = sh_remaining;
-    }
-    KthResult r;
-    r.key = prefix;
-    r.take_eq = remaining;
-    r.eq_count = (long long)sh_bin_count;
-    __syncthreads();  // the shared results may be rewritten by a later call
-    return r;
 }
 
 // ---------------------------------------------------------------- cluster form
@@ -256,52 +135,26 @@ __device__ __forceinline__ int cblock_exclusive_scan(int v, int* warp_buf, int& 
     return before + x - v;
 }
 
-__global__ void __launch_bounds__(kCThreads)
-    select_cluster_kernel(const float* __restrict__ gate, const int32_t* __restrict__ cu_seqlens, int nseq, int L,
-                          double ratio, int32_t* __restrict__ sel_idx, int32_t* __restrict__ cu_sel, int resident_cap)
+struct ClusterKth {
+    uint32_t key;        // the k-th largest key of the cluster's keys
+    long long take_eq;   // how many keys equal to it are among the k largest
+    long long eq_count;  // how many keys equal to it there are
+};
+
+// Radix select over the keys of all CTAs of the cluster (this CTA's slice: key_at(i), i < n)
+// with four 8-bit passes, 1 <= k <= the cluster's key count.  Called by every thread of every
+// CTA of the cluster with the same k.  Each pass counts the slice into a shared-memory
+// histogram; after a cluster barrier every CTA sums the cluster's histograms through
+// distributed shared memory and takes the same digit.  The caller passes one more cluster
+// barrier before its CTA exits, so no CTA leaves while another still reads its histograms.
+template <typename KeyAt>
+__device__ ClusterKth cluster_kth_largest(KeyAt key_at, long long n, long long k, uint32_t nranks)
 {
-    extern __shared__ uint32_t slice_keys[];  // resident_cap keys (at most kSliceResident)
-    __shared__ uint32_t hist[2][256];         // this slice's counts, alternating between passes
-    __shared__ uint32_t tot[256];             // the cluster's counts
-    __shared__ long long cnt[2];              // keys of this slice above T, equal to T
-    __shared__ int warp_buf[32];
+    __shared__ uint32_t hist[2][256];  // this slice's counts, alternating between passes
+    __shared__ uint32_t tot[256];      // the cluster's counts
     __shared__ uint32_t sh_digit, sh_bin_count;
-    __shared__ long long sh_remaining, sh_sel_before, sh_eq_quota;
-
-    const uint32_t rank = cluster_ctarank();
-    const uint32_t nranks = cluster_nctarank();  // the launch's cluster size, 1 to kClusterCtas
-    const int s = blockIdx.y;
+    __shared__ long long sh_remaining;
     const int tid = threadIdx.x;
-    long long start, len, out_off;
-    if (cu_seqlens) {
-        start = cu_seqlens[s];
-        len = (long long)cu_seqlens[s + 1] - start;
-        out_off = 0;
-        for (int t = 0; t < s; ++t) out_off += budget_count(ratio, (long long)cu_seqlens[t + 1] - cu_seqlens[t]);
-    } else {
-        start = (long long)s * L;
-        len = L;
-        out_off = (long long)s * budget_count(ratio, L);
-    }
-    const long long k = budget_count(ratio, len);  // the same in every CTA of the cluster
-    if (rank == 0 && tid == 0) {
-        cu_sel[s + 1] = (int32_t)(out_off + k);
-        if (s == 0) cu_sel[0] = 0;
-    }
-    if (k <= 0) return;
-    const long long lo = len * rank / nranks, hi = len * (rank + 1) / nranks, n = hi - lo;
-    const float* g = gate + start + lo;
-    int32_t* out = sel_idx + out_off;
-    if (k == len) {
-        for (long long i = tid; i < n; i += kCThreads) out[lo + i] = (int32_t)(lo + i);
-        return;
-    }
-    const bool resident = n <= resident_cap;  // the launch sized the array for the longest sequence
-    if (resident)
-        for (long long i = tid; i < n; i += kCThreads) slice_keys[i] = gate_key(__ldg(g + i));
-    auto key_at = [&](long long i) -> uint32_t { return resident ? slice_keys[i] : gate_key(__ldg(g + i)); };
-
-    // ---- radix select of the k-th largest key over the whole sequence
     uint32_t prefix = 0, mask = 0;
     long long remaining = k;
     for (int pass = 0; pass < 4; ++pass) {
@@ -357,9 +210,61 @@ __global__ void __launch_bounds__(kCThreads)
         mask |= 255u << shift;
         remaining = sh_remaining;
     }
-    const uint32_t T = prefix;                    // the k-th largest key
-    const long long take_eq = remaining;          // how many keys equal to T are selected
-    const bool all_eq = take_eq == (long long)sh_bin_count;
+    ClusterKth r;
+    r.key = prefix;
+    r.take_eq = remaining;
+    r.eq_count = (long long)sh_bin_count;
+    __syncthreads();
+    return r;
+}
+
+__global__ void __launch_bounds__(kCThreads)
+    select_cluster_kernel(const float* __restrict__ gate, const int32_t* __restrict__ cu_seqlens, int nseq, int L,
+                          double ratio, int32_t* __restrict__ sel_idx, int32_t* __restrict__ cu_sel, int resident_cap)
+{
+    extern __shared__ uint32_t slice_keys[];  // resident_cap keys (at most kSliceResident)
+    __shared__ long long cnt[2];              // keys of this slice above T, equal to T
+    __shared__ int warp_buf[32];
+    __shared__ long long sh_sel_before, sh_eq_quota;
+
+    const uint32_t rank = cluster_ctarank();
+    const uint32_t nranks = cluster_nctarank();  // the launch's cluster size, 1 to kClusterCtas
+    const int s = blockIdx.y;
+    const int tid = threadIdx.x;
+    long long start, len, out_off;
+    if (cu_seqlens) {
+        start = cu_seqlens[s];
+        len = (long long)cu_seqlens[s + 1] - start;
+        out_off = 0;
+        for (int t = 0; t < s; ++t) out_off += budget_count(ratio, (long long)cu_seqlens[t + 1] - cu_seqlens[t]);
+    } else {
+        start = (long long)s * L;
+        len = L;
+        out_off = (long long)s * budget_count(ratio, L);
+    }
+    const long long k = budget_count(ratio, len);  // the same in every CTA of the cluster
+    if (rank == 0 && tid == 0) {
+        cu_sel[s + 1] = (int32_t)(out_off + k);
+        if (s == 0) cu_sel[0] = 0;
+    }
+    if (k <= 0) return;
+    const long long lo = len * rank / nranks, hi = len * (rank + 1) / nranks, n = hi - lo;
+    const float* g = gate + start + lo;
+    int32_t* out = sel_idx + out_off;
+    if (k == len) {
+        for (long long i = tid; i < n; i += kCThreads) out[lo + i] = (int32_t)(lo + i);
+        return;
+    }
+    const bool resident = n <= resident_cap;  // the launch sized the array for the longest sequence
+    if (resident)
+        for (long long i = tid; i < n; i += kCThreads) slice_keys[i] = gate_key(__ldg(g + i));
+    auto key_at = [&](long long i) -> uint32_t { return resident ? slice_keys[i] : gate_key(__ldg(g + i)); };
+
+    // ---- radix select of the k-th largest key over the whole sequence
+    const ClusterKth kr = cluster_kth_largest(key_at, n, k, nranks);
+    const uint32_t T = kr.key;                    // the k-th largest key
+    const long long take_eq = kr.take_eq;         // how many keys equal to T are selected
+    const bool all_eq = take_eq == kr.eq_count;
 
     // ---- this slice's keys above and equal to T, then its place among the cluster's slices
     int n_gt = 0, n_eq = 0;
@@ -452,61 +357,97 @@ __device__ __forceinline__ void seq_span(const int32_t* cu_seqlens, int L, int s
     }
 }
 
-// Per sequence: how many logits lie above the threshold.
-__global__ void __launch_bounds__(kSelThreads) threshold_count_kernel(const float* __restrict__ gate,
-                                                                     const int32_t* __restrict__ cu_seqlens, int L,
-                                                                     const float* __restrict__ tau,
-                                                                     int32_t* __restrict__ counts)
+__device__ __forceinline__ float key_to_float(uint32_t key)
+{
+    if (key == 0u) return __int_as_float(0x7fc00000);  // NaN
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// The threshold rule and the controller step on clusters of CTAs: a sequence (for the
+// controller, the whole batch) in contiguous slices exactly as in the top-k selection above.
+
+// Slice count of logits above the threshold, summed over the cluster into counts[s].
+__global__ void __launch_bounds__(kCThreads) threshold_count_cluster_kernel(const float* __restrict__ gate,
+                                                                           const int32_t* __restrict__ cu_seqlens,
+                                                                           int L, const float* __restrict__ tau,
+                                                                           int32_t* __restrict__ counts)
 {
     __shared__ int warp_buf[32];
+    __shared__ long long slice_count;
+    const uint32_t rank = cluster_ctarank(), nranks = cluster_nctarank();
+    const int s = blockIdx.y;
     long long start, len;
-    seq_span(cu_seqlens, L, blockIdx.x, start, len);
+    seq_span(cu_seqlens, L, s, start, len);
+    const long long lo = len * rank / nranks, hi = len * (rank + 1) / nranks;
     const float t = *tau;
     const bool tau_nan = isnan(t);
     const uint32_t tkey = gate_key(t);
     int c = 0;
-    for (long long i = threadIdx.x; i < len; i += kSelThreads) c += above(gate_key(__ldg(gate + start + i)), tkey, tau_nan);
+    for (long long i = lo + threadIdx.x; i < hi; i += kCThreads) c += above(gate_key(__ldg(gate + start + i)), tkey, tau_nan);
     int total;
-    block_exclusive_scan(c, warp_buf, total);
-    if (threadIdx.x == 0) counts[blockIdx.x] = total;
+    cblock_exclusive_scan(c, warp_buf, total);
+    if (threadIdx.x == 0) slice_count = total;
+    cluster_sync_all();
+    if (rank == 0 && threadIdx.x == 0) {
+        long long sum = 0;
+        for (uint32_t r = 0; r < nranks; ++r) sum += ld_cluster_s64(cluster_map(&slice_count, r));
+        counts[s] = (int32_t)sum;
+    }
+    cluster_sync_all();  // no CTA leaves while rank 0 still reads its count
 }
 
-// Per sequence: the positions above the threshold, ascending, at most `cap` of them,
-// written at the sequence's offset (the capped counts of the earlier sequences).
-__global__ void __launch_bounds__(kSelThreads) threshold_compact_kernel(
+// Per sequence: the positions above the threshold, ascending, at most `cap` of them, written at
+// the sequence's offset (the capped counts of the earlier sequences); each slice after the
+// positions of the lower-ranked slices.
+__global__ void __launch_bounds__(kCThreads) threshold_compact_cluster_kernel(
     const float* __restrict__ gate, const int32_t* __restrict__ cu_seqlens, int L, const float* __restrict__ tau,
     int cap, const int32_t* __restrict__ counts, int32_t* __restrict__ sel_idx, int32_t* __restrict__ cu_sel,
     uint32_t* status)
 {
     __shared__ int warp_buf[32];
-    const int s = blockIdx.x;
+    __shared__ long long slice_count, sh_before;
+    const uint32_t rank = cluster_ctarank(), nranks = cluster_nctarank();
+    const int s = blockIdx.y;
     long long start, len;
     seq_span(cu_seqlens, L, s, start, len);
     long long off = 0;
     for (int t = 0; t < s; ++t) off += min(counts[t], cap);
     const int mine = min(counts[s], cap);
-    if (threadIdx.x == 0) {
+    if (rank == 0 && threadIdx.x == 0) {
         cu_sel[s + 1] = (int32_t)(off + mine);
         if (s == 0) cu_sel[0] = 0;
         if (counts[s] > cap) atomicOr(status, kStatusCapacity);
     }
-    if (mine == 0) return;
+    if (mine == 0) return;  // the same in every CTA of the cluster
+    const long long lo = len * rank / nranks, hi = len * (rank + 1) / nranks;
     const float t = *tau;
     const bool tau_nan = isnan(t);
     const uint32_t tkey = gate_key(t);
+    int c = 0;
+    for (long long i = lo + threadIdx.x; i < hi; i += kCThreads) c += above(gate_key(__ldg(gate + start + i)), tkey, tau_nan);
+    int total;
+    cblock_exclusive_scan(c, warp_buf, total);
+    if (threadIdx.x == 0) slice_count = total;
+    cluster_sync_all();
+    if (threadIdx.x == 0) {
+        long long before = 0;
+        for (uint32_t r = 0; r < rank; ++r) before += ld_cluster_s64(cluster_map(&slice_count, r));
+        sh_before = before;
+    }
+    __syncthreads();
     int32_t* out = sel_idx + off;
-    long long written = 0;
-    for (long long chunk = 0; chunk < len && written < mine; chunk += (long long)kSelThreads * kItems) {
+    long long written = sh_before;
+    for (long long chunk = lo; chunk < hi && written < mine; chunk += (long long)kCThreads * kItems) {
         const long long i0 = chunk + (long long)threadIdx.x * kItems;
         bool sel[kItems];
         int n_sel = 0;
         #pragma unroll
         for (int u = 0; u < kItems; ++u) {
-            sel[u] = (i0 + u < len) && above(gate_key(__ldg(gate + start + i0 + u)), tkey, tau_nan);
+            sel[u] = (i0 + u < hi) && above(gate_key(__ldg(gate + start + i0 + u)), tkey, tau_nan);
             n_sel += sel[u] ? 1 : 0;
         }
-        int total;
-        const int before = block_exclusive_scan(n_sel, warp_buf, total);
+        int chunk_total;
+        const int before = cblock_exclusive_scan(n_sel, warp_buf, chunk_total);
         int o = 0;
         #pragma unroll
         for (int u = 0; u < kItems; ++u) {
@@ -515,39 +456,37 @@ __global__ void __launch_bounds__(kSelThreads) threshold_compact_kernel(
                 if (dst < mine) out[dst] = (int32_t)(i0 + u);
             }
         }
-        written += total;
+        written += chunk_total;
     }
+    cluster_sync_all();  // no CTA leaves while a higher rank still reads its count
 }
 
-__device__ __forceinline__ float key_to_float(uint32_t key)
+// The controller step over the whole batch (all n valid logits): target q = the (k+1)-th
+// largest logit, k = budget_count(ratio, n) (-inf when k = n, or when that place holds a NaN);
+// tau <- tau + beta * (q - tau) in fp32 with a rounding after each operation, or tau <- q when
+// either is not finite.  The batch is spread over the cluster in contiguous slices.
+__global__ void __launch_bounds__(kCThreads) threshold_update_cluster_kernel(
+    const float* __restrict__ gate, const int32_t* __restrict__ cu_seqlens, int nseq, long long n_fixed, double ratio,
+    float beta, float* __restrict__ tau, float* __restrict__ target_out, int resident_cap)
 {
-    if (key == 0u) return __int_as_float(0x7fc00000);  // NaN
-    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
-}
-
-// The controller step over the whole batch (all n valid logits): target q = the
-// (k+1)-th largest logit, k = budget_count(ratio, n) (-inf when k = n, or when
-// that place holds a NaN); tau <- tau + beta * (q - tau) in fp32 with a rounding
-// after each operation, or tau <- q when either is not finite.
-__global__ void __launch_bounds__(kSelThreads) threshold_update_kernel(const float* __restrict__ gate,
-                                                                      const int32_t* __restrict__ cu_seqlens,
-                                                                      int nseq, long long n_fixed, double ratio,
-                                                                      float beta, float* __restrict__ tau,
-                                                                      float* __restrict__ target_out)
-{
-    extern __shared__ uint32_t dyn_smem[];
-    uint32_t* whist = dyn_smem;  // [kSelWarps][256]
-    __shared__ uint32_t hist[256];
-    const long long n = cu_seqlens ? (long long)cu_seqlens[nseq] : n_fixed;
-    const long long k = budget_count(ratio, n);
+    extern __shared__ uint32_t slice_keys[];  // resident_cap keys
+    const uint32_t rank = cluster_ctarank(), nranks = cluster_nctarank();
+    const long long n_all = cu_seqlens ? (long long)cu_seqlens[nseq] : n_fixed;
+    const long long k = budget_count(ratio, n_all);
     float q = -INFINITY;
-    if (k < n) {
-        auto key_at = [&](long long i) -> uint32_t { return gate_key(__ldg(gate + i)); };
-        const KthResult r = radix_kth_largest(key_at, n, k + 1, whist, hist);
+    if (k < n_all) {  // the same in every CTA of the cluster
+        const long long lo = n_all * rank / nranks, hi = n_all * (rank + 1) / nranks, n = hi - lo;
+        const float* g = gate + lo;
+        const bool resident = n <= resident_cap;
+        if (resident)
+            for (long long i = threadIdx.x; i < n; i += kCThreads) slice_keys[i] = gate_key(__ldg(g + i));
+        auto key_at = [&](long long i) -> uint32_t { return resident ? slice_keys[i] : gate_key(__ldg(g + i)); };
+        const ClusterKth r = cluster_kth_largest(key_at, n, k + 1, nranks);
         q = key_to_float(r.key);
         if (isnan(q)) q = -INFINITY;
+        cluster_sync_all();  // no CTA leaves while another still reads its histograms
     }
-    if (threadIdx.x == 0) {
+    if (rank == 0 && threadIdx.x == 0) {
         const float t = *tau;
         const bool finite = isfinite(t) && isfinite(q);
         *tau = finite ? __fadd_rn(t, __fmul_rn(beta, __fsub_rn(q, t))) : q;
@@ -555,45 +494,17 @@ __global__ void __launch_bounds__(kSelThreads) threshold_update_kernel(const flo
     }
 }
 
-}  // namespace
-
-cudaError_t launch_threshold_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, const float* tau,
-                                    int max_selected, int32_t* counts, int32_t* sel_idx, int32_t* cu_sel,
-                                    uint32_t* status, cudaStream_t stream)
+// CTAs per cluster for `n` keys: one per kKeysPerCta, a power of two, at most kClusterCtas.
+int cluster_ctas_for(long long n)
 {
-    if (nseq <= 0) return cudaSuccess;
-    threshold_count_kernel<<<nseq, kSelThreads, 0, stream>>>(gate, cu_seqlens, L, tau, counts);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    threshold_compact_kernel<<<nseq, kSelThreads, 0, stream>>>(gate, cu_seqlens, L, tau, max_selected, counts,
-                                                               sel_idx, cu_sel, status);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_threshold_update(const float* gate, const int32_t* cu_seqlens, int nseq, long long n_fixed,
-                                    double ratio, float beta, float* tau, float* target_out, cudaStream_t stream)
-{
-    const size_t smem = (size_t)kSelWarps * 256 * 4;
-    threshold_update_kernel<<<1, kSelThreads, smem, stream>>>(gate, cu_seqlens, nseq, n_fixed, ratio, beta, tau,
-                                                              target_out);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, int max_len,
-                          double ratio, int32_t* sel_idx, int32_t* cu_sel, cudaStream_t stream)
-{
-    if (nseq <= 0) return cudaSuccess;
-    // One cluster per sequence, of one CTA per kKeysPerCta keys of the longest sequence (a power
-    // of two, at most kClusterCtas); its slices of at most kSliceResident keys stay in shared
-    // memory.
-    const long long ml = max_len > 0 ? max_len : 1;
     int ctas = 1;
-    while (ctas < kClusterCtas && (long long)ctas * kKeysPerCta < ml) ctas *= 2;
-    const long long slice = (ml + ctas - 1) / ctas;
-    const int cap = (int)(slice < kSliceResident ? slice : kSliceResident);
-    const size_t smem = (size_t)cap * 4;
-    cudaError_t e = cudaFuncSetAttribute(select_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    while (ctas < kClusterCtas && (long long)ctas * kKeysPerCta < n) ctas *= 2;
+    return ctas;
+}
+
+template <typename... Args, typename... Act>
+cudaError_t launch_cluster(void (*kern)(Args...), int ctas, int nseq, size_t smem, cudaStream_t stream, Act&&... args)
+{
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(ctas, nseq);
     cfg.blockDim = dim3(kCThreads);
@@ -606,7 +517,57 @@ cudaError_t launch_select(const float* gate, const int32_t* cu_seqlens, int nseq
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, select_cluster_kernel, gate, cu_seqlens, nseq, L, ratio, sel_idx, cu_sel, cap);
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Act>(args)...);
+}
+
+}  // namespace
+
+cudaError_t launch_threshold_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, int max_len,
+                                    const float* tau, int max_selected, int32_t* counts, int32_t* sel_idx,
+                                    int32_t* cu_sel, uint32_t* status, cudaStream_t stream)
+{
+    if (nseq <= 0) return cudaSuccess;
+    const int ctas = cluster_ctas_for(max_len > 0 ? max_len : 1);
+    cudaError_t e = launch_cluster(threshold_count_cluster_kernel, ctas, nseq, 0, stream, gate, cu_seqlens, L, tau,
+                                   counts);
+    if (e != cudaSuccess) return e;
+    return launch_cluster(threshold_compact_cluster_kernel, ctas, nseq, 0, stream, gate, cu_seqlens, L, tau,
+                          max_selected, (const int32_t*)counts, sel_idx, cu_sel, status);
+}
+
+cudaError_t launch_threshold_update(const float* gate, const int32_t* cu_seqlens, int nseq, long long n_all,
+                                    long long n_fixed, double ratio, float beta, float* tau, float* target_out,
+                                    cudaStream_t stream)
+{
+    // n_all: the number of logits of the batch as the host knows it (B * L, or the packed
+    // total), which sizes the cluster; the kernel reads the packed total from cu_seqlens.
+    const int ctas = cluster_ctas_for(n_all > 0 ? n_all : 1);
+    const long long slice = ((n_all > 0 ? n_all : 1) + ctas - 1) / ctas;
+    const int cap = (int)(slice < kSliceResident ? slice : kSliceResident);
+    const size_t smem = (size_t)cap * 4;
+    cudaError_t e =
+        cudaFuncSetAttribute(threshold_update_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_cluster(threshold_update_cluster_kernel, ctas, 1, smem, stream, gate, cu_seqlens, nseq, n_fixed,
+                          ratio, beta, tau, target_out, cap);
+}
+
+cudaError_t launch_select(const float* gate, const int32_t* cu_seqlens, int nseq, int L, int max_len,
+                          double ratio, int32_t* sel_idx, int32_t* cu_sel, cudaStream_t stream)
+{
+    if (nseq <= 0) return cudaSuccess;
+    // One cluster per sequence, of one CTA per kKeysPerCta keys of the longest sequence (a power
+    // of two, at most kClusterCtas); its slices of at most kSliceResident keys stay in shared
+    // memory.
+    const long long ml = max_len > 0 ? max_len : 1;
+    const int ctas = cluster_ctas_for(ml);
+    const long long slice = (ml + ctas - 1) / ctas;
+    const int cap = (int)(slice < kSliceResident ? slice : kSliceResident);
+    const size_t smem = (size_t)cap * 4;
+    cudaError_t e = cudaFuncSetAttribute(select_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_cluster(select_cluster_kernel, ctas, nseq, smem, stream, gate, cu_seqlens, nseq, L, ratio, sel_idx,
+                          cu_sel, cap);
 }
 
 }  // namespace logo
