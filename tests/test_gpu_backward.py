@@ -33,10 +33,16 @@ def close(got, ref, what):
     assert torch.isfinite(got).all(), f"{what}: non-finite values"
     scale = ref.abs().max().item()
     err = (got - ref).abs().max().item()
+    if scale == 0.0:
+        # An exactly zero gradient (W = 1 with no selected rows: every dS = P (dP - D) with
+        # P = 1 and dP = D) comes out of the kernels as the fp32 rounding difference of two
+        # sums of O(1) products, dP by the tensor cores and D by the prep kernel.
+        print(f"{what}: exact zero in the reference, max-abs {err:.3e}")
+        assert err <= 1e-4, f"{what}: {err:.3e} where the gradient is exactly zero"
+        return
     rel = ((got - ref).norm() / ref.norm().clamp_min(1e-30)).item()
     print(f"{what}: max-abs {err:.3e} (ref max {scale:.3e}) rel-L2 {rel:.3e}")
-    assert rel <= REL_L2 and err <= MAX_ABS_FRAC * max(scale, 1e-30), \
-        f"{what}: max-abs {err:.3e} of {scale:.3e}, rel-L2 {rel:.3e}"
+    assert rel <= REL_L2 and err <= MAX_ABS_FRAC * scale, f"{what}: max-abs {err:.3e} of {scale:.3e}, rel-L2 {rel:.3e}"
 
 
 def gpu_run(w, e):

@@ -141,13 +141,15 @@ def test_forward_running_max_growth(case):
     few keys carry a large norm (spikes: every 97th key x12), so the maximum
     keeps growing by many powers of two from tile to tile.
 
-    Outputs here reach |o| ~ 8, where one bf16 rounding alone is up to 2^-6
-    (0.016) and the merged output is rounded twice (the local branch is stored
-    in bf16 and read back by the merge), so an absolute 2e-2 bound is finer
-    than the output format at that magnitude (a CPU emulation of the rounding
-    steps alone gives 0.021 to 0.027).  The max-abs bound is therefore scaled
-    with the output: 2e-2 * max(1, max|ref| / 4), i.e. 2e-2 at the magnitude
-    of N(0,1) outputs; the relative-L2 bound stays 5e-3.
+    Outputs here reach |o| ~ 8.  A bf16 value in [2^e, 2^(e+1)) is rounded by up
+    to half its spacing 2^(e-7), and the merged output is rounded twice (the
+    local branch is stored in bf16 and read back by the merge), so the format
+    alone allows up to 2^(e-7) at that magnitude: 0.031 for |o| in [4, 8), more
+    than an absolute 2e-2 (a CPU emulation of the rounding steps alone gives
+    0.021 to 0.027 on these inputs).  The max-abs bound is therefore scaled with
+    the output: 2e-2 * max(1, max|ref| / 2), which stays above 2^(e-7) for every
+    e >= 1 and is 2e-2 at the magnitude of N(0,1) outputs; the relative-L2 bound
+    stays 5e-3.
     """
     name, B, Hq, Hkv, L, d, W, ratio, kind = case
     w = workloads.make(B, Hq, Hkv, L, d, W, ratio, seed=5, qkv_scale=1.0, name=name)
@@ -166,7 +168,7 @@ def test_forward_running_max_growth(case):
     loc = logo.local_attn(q, k, v, w.W, ws)
     logo.check(ws)
     for got, r, what in ((loc, ref["local"], "local"), (out, ref["out"], "merged")):
-        bound = MAX_ABS * max(1.0, r.abs().max().item() / 4.0)
+        bound = MAX_ABS * max(1.0, r.abs().max().item() / 2.0)
         close(got, r, what, max_abs=bound)
 
 

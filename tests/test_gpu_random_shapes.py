@@ -53,15 +53,17 @@ def test_forward_random_shape(seed):
     ref = oracle.forward(w.q, w.k, w.v, w.g, w.W, w.ratio, cu_seqlens=w.cu_seqlens)
     assert sel_lists(sel, cu_sel) == oracle_sel_lists(w)
     T = w.L if w.cu_seqlens is None else int(w.cu_seqlens[-1])
-    # Unscaled N(0,1) inputs with a short window give outputs up to |o| ~ 8, where one bf16
-    # rounding is up to 2^-6 and the merged row is rounded twice: the max-abs bound scales with
-    # the output as in the large-output tests, 2e-2 * max(1, max|ref| / 4); rel-L2 stays 5e-3.
+    # Unscaled N(0,1) inputs with a short window give outputs up to |o| ~ 8; the merged row is
+    # rounded to bf16 twice, up to one bf16 spacing at its magnitude: the max-abs bound scales
+    # with the output as in the large-output tests, 2e-2 * max(1, max|ref| / 2); rel-L2 5e-3.
     r = ref["out"][:, :, :T]
     close(out[:, :, :T], r, f"random {seed} {(B, Hq, Hkv, L, d, W, ratio, lens)}",
-          max_abs=MAX_ABS * max(1.0, r.abs().max().item() / 4.0))
+          max_abs=MAX_ABS * max(1.0, r.abs().max().item() / 2.0))
 
 
-@pytest.mark.parametrize("seed", CASES[:12])
+# seeds 120 and 184 draw W = 1 with ratio 0: every row attends to itself alone, so dQ is exactly
+# zero (the one softmax weight is 1 and dP equals D)
+@pytest.mark.parametrize("seed", CASES[:12] + [120, 184])
 def test_backward_random_shape(seed):
     from tests.test_gpu_backward import close as close_grad, gpu_run
 
@@ -100,4 +102,4 @@ def test_forward_medium_edge_groups(case):
     assert sel_lists(sel, cu_sel) == oracle_sel_lists(w)
     T = w.L if w.cu_seqlens is None else int(w.cu_seqlens[-1])
     r = ref["out"][:, :, :T]
-    close(out[:, :, :T], r, name, max_abs=MAX_ABS * max(1.0, r.abs().max().item() / 4.0))
+    close(out[:, :, :T], r, name, max_abs=MAX_ABS * max(1.0, r.abs().max().item() / 2.0))
