@@ -62,8 +62,9 @@ def test_forward_random_shape(seed):
 
 
 # seeds 120 and 184 draw W = 1 with ratio 0: every row attends to itself alone, so dQ is exactly
-# zero (the one softmax weight is 1 and dP equals D)
-@pytest.mark.parametrize("seed", CASES[:12] + [120, 184])
+# zero (the one softmax weight is 1 and dP equals D); seed 360 selects one row of a 5-token
+# sequence whose gate gradient sums terms that largely cancel
+@pytest.mark.parametrize("seed", CASES[:12] + [120, 184, 360])
 def test_backward_random_shape(seed):
     from tests.test_gpu_backward import close as close_grad, gpu_run
 
@@ -78,7 +79,25 @@ def test_backward_random_shape(seed):
     close_grad(dk[:, :, :T], ref["dk"][:, :, :T], what + " dk")
     close_grad(dv[:, :, :T], ref["dv"][:, :, :T], what + " dv")
     if (ref["dg"] != 0).any():
-        close_grad(dg[:, :T], ref["dg"][:, :T], what + " dgate")
+        check_dgate(w, e, dg[:, :T], ref["dg"][:, :T], T, what + " dgate")
+
+
+def check_dgate(w, e, dg, ref_dg, T, what):
+    """The gate gradient of a selected row is sigma'(g) * sum over heads and columns of
+    dout * global (the global branch before the gate).  The kernels form it from the bf16 global
+    branch, so its error is bounded by the rounding of the terms, not by the size of the sum:
+    where the terms cancel the relative error of the sum grows without bound.  The check is the
+    dot product's forward-error bound with 5e-3 (about 2.5 bf16 roundings) per term:
+    |dg - ref| <= 5e-3 * sigma'(g) * sum |dout * global|, row by row."""
+    fwd = oracle.forward(w.q, w.k, w.v, w.g, w.W, w.ratio, cu_seqlens=w.cu_seqlens, want_branches=True)
+    glob = fwd["global"][:, :, :T]
+    terms = (e[:, :, :T].double() * glob).abs().sum(dim=(1, 3))  # [B, T]
+    sg = torch.sigmoid(w.g[:, :T].double())
+    bound = 5e-3 * sg * (1.0 - sg) * terms
+    err = (dg.double().cpu() - ref_dg.double()).abs()
+    worst = (err - bound).max().item()
+    print(f"{what}: max-abs {err.max().item():.3e}, worst margin {worst:.3e}")
+    assert (err <= bound + 1e-7).all(), f"{what}: an error above the per-row bound (margin {worst:.3e})"
 
 
 MEDIUM = [
