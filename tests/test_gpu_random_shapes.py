@@ -122,3 +122,35 @@ def test_forward_medium_edge_groups(case):
     T = w.L if w.cu_seqlens is None else int(w.cu_seqlens[-1])
     r = ref["out"][:, :, :T]
     close(out[:, :, :T], r, name, max_abs=MAX_ABS * max(1.0, r.abs().max().item() / 2.0))
+
+
+def draw_medium(seed):
+    """A seeded shape of a few thousand tokens: group sizes 1 to 8, d 64 or 128, windows from 64
+    to 8192 and ratios from 0.02 to 1, fixed-length batches or 2 to 5 packed sequences."""
+    rng = random.Random(5000 + seed)
+    Hkv = rng.choice([1, 2])
+    G = rng.choice([1, 2, 3, 4, 6, 8])
+    d = rng.choice([64, 128])
+    W = rng.choice([64, 500, 1024, 2047, 4096, 8192])
+    ratio = rng.choice([0.02, 0.1, 0.2, 0.33, 0.6, 1.0])
+    if rng.random() < 0.4:
+        seqlens = [rng.randrange(1, 6000) for _ in range(rng.randrange(2, 6))]
+        return 1, Hkv * G, Hkv, 0, d, W, ratio, seqlens
+    return rng.choice([1, 2]), Hkv * G, Hkv, rng.randrange(1000, 9000), d, W, ratio, None
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_forward_medium_random_shape(seed):
+    """Every element at sizes that span many CTAs of both launches and ragged tails."""
+    B, Hq, Hkv, L, d, W, ratio, lens = draw_medium(seed)
+    w = workloads.make(B, Hq, Hkv, L, d, W, ratio, seed=seed, seqlens=lens, name=f"medium{seed}")
+    q, k, v, g, cu = to_dev(w)
+    ml = max(w.seqlens)
+    out, sel, cu_sel = logo.forward(q, k, v, g, w.W, w.ratio, cu_seqlens=cu, max_seqlen=ml if cu is not None else None)
+    torch.cuda.synchronize()
+    ref = oracle.forward(w.q, w.k, w.v, w.g, w.W, w.ratio, cu_seqlens=w.cu_seqlens)
+    assert sel_lists(sel, cu_sel) == oracle_sel_lists(w)
+    T = w.L if w.cu_seqlens is None else int(w.cu_seqlens[-1])
+    r = ref["out"][:, :, :T]
+    close(out[:, :, :T], r, f"medium {seed} {(B, Hq, Hkv, L, d, W, ratio, lens)}",
+          max_abs=MAX_ABS * max(1.0, r.abs().max().item() / 2.0))
