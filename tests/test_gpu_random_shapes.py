@@ -154,3 +154,36 @@ def test_forward_medium_random_shape(seed):
     r = ref["out"][:, :, :T]
     close(out[:, :, :T], r, f"medium {seed} {(B, Hq, Hkv, L, d, W, ratio, lens)}",
           max_abs=MAX_ABS * max(1.0, r.abs().max().item() / 2.0))
+
+
+def draw_medium_backward(seed):
+    """A seeded shape of 500 to 3000 tokens for the backward: group sizes 1 to 8, d 64 or 128,
+    windows 64 to 4096, ratios 0.05 to 1, fixed-length batches or 2 to 4 packed sequences."""
+    rng = random.Random(7000 + seed)
+    Hkv = rng.choice([1, 2])
+    G = rng.choice([1, 2, 3, 4, 8])
+    d = rng.choice([64, 128])
+    W = rng.choice([64, 300, 1024, 4096])
+    ratio = rng.choice([0.05, 0.2, 0.5, 1.0])
+    if rng.random() < 0.4:
+        return 1, Hkv * G, Hkv, 0, d, W, ratio, [rng.randrange(1, 2500) for _ in range(rng.randrange(2, 5))]
+    return rng.choice([1, 2]), Hkv * G, Hkv, rng.randrange(500, 3000), d, W, ratio, None
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_backward_medium_random_shape(seed):
+    """Every gradient element at sizes that span many CTAs of the dQ and dK/dV launches."""
+    from tests.test_gpu_backward import close as close_grad, gpu_run
+
+    B, Hq, Hkv, L, d, W, ratio, lens = draw_medium_backward(seed)
+    w = workloads.make(B, Hq, Hkv, L, d, W, ratio, seed=seed, seqlens=lens, name=f"bmedium{seed}")
+    e = torch.randn(w.q.shape, generator=torch.Generator().manual_seed(seed)).bfloat16()
+    dq, dk, dv, dg = gpu_run(w, e)
+    ref = oracle.backward(w.q, w.k, w.v, w.g, e, w.W, w.ratio, cu_seqlens=w.cu_seqlens)
+    T = w.L if w.cu_seqlens is None else int(w.cu_seqlens[-1])
+    what = f"medium backward {seed} {(B, Hq, Hkv, L, d, W, ratio, lens)}"
+    close_grad(dq[:, :, :T], ref["dq"][:, :, :T], what + " dq")
+    close_grad(dk[:, :, :T], ref["dk"][:, :, :T], what + " dk")
+    close_grad(dv[:, :, :T], ref["dv"][:, :, :T], what + " dv")
+    if (ref["dg"] != 0).any():
+        check_dgate(w, e, dg[:, :T], ref["dg"][:, :T], T, what + " dgate")
